@@ -1,0 +1,156 @@
+/*
+ * vdn.h - C ABI of the B200 (sm_100a) forward pass of VideoDeltaNet's hybrid
+ * attention layer (VDN-MiniMax-H3).
+ *
+ * The layer, as the pages describe it:
+ *  - latent frames are grouped into blocks of 5 consecutive frames; a block
+ *    attends exactly (softmax) with itself and its two neighbouring blocks,
+ *    and the first and last frames are boundary anchors visible to every
+ *    block ["VDN-MiniMax-H3" (openi.cn), section 技术原理：局部精确、远程压缩;
+ *    "VDN-MiniMax-H3 - OpenVDN's Open-Source Video Generation Acceleration
+ *    Solution" (nav.superapi.store), Technical Principles, Local Softmax
+ *    Branch];
+ *  - text tokens are visible to every frame in the softmax branch and are
+ *    written once into the linear state at initialisation [nav.superapi.store
+ *    page, Technical Principles, Text Dual-Branch Injection];
+ *  - Video Delta Attention (VDA): one joint normal-equation solve per frame
+ *    replaces the token-by-token delta rule [nav.superapi.store page,
+ *    Technical Principles, Video Delta Attention];
+ *  - the linear branch sums the context before and after the current window,
+ *    leaving out the window frames and the anchors [openi.cn page, same
+ *    section];
+ *  - each branch has a content-dependent sigmoid gate and the linear output
+ *    is RMS-normalised before its gate [openi.cn page, same section, last
+ *    paragraph; nav.superapi.store page, Gated Fusion Mechanism].
+ *
+ * The pages print no formulas; this library implements one fixed reading:
+ *   o_soft = softmax(q K^T / sqrt(d)) V over the keys of frames in
+ *            {window of the query's block} U {0, F-1} and all text tokens;
+ *   k_hat  = k / max(||k||_2, 1e-12)  (VDA only, video and text keys);
+ *   S_text = (lambda I + Kt^T Kt)^-1 Kt^T Vt;
+ *   S_f    = (lambda I + K_f^T K_f)^-1 (lambda S_prev + K_f^T V_f);
+ *   forward scan over frames 1..F-2 and backward scan over F-2..1, both
+ *   starting from S_text; block b reads R_b = Sfwd[max(w0-1,0)] +
+ *   Sbwd[min(w1+1,F-1)] where [w0, w1] is its window, Sfwd[0] = Sbwd[F-1] =
+ *   S_text; o_lin = q^T R_b;
+ *   out = sigmoid(g_s) o_soft + sigmoid(g_l) * w_h * o_lin / sqrt(mean(o_lin^2) + eps).
+ *
+ * Conventions for every entry point
+ *  - Token-major packed layouts, row-major and contiguous:
+ *      q, k, v, out, o_soft : [N, H, d]       (N = off_host[F])
+ *      kt, vt               : [T, H, d]
+ *      g_s, g_l             : [N, H]
+ *      rms_w                : [H, d] fp32
+ *      states               : [.., H, d, d] fp32, S[key dim][value dim]
+ *    Element type of q, k, v, kt, vt, g_s, g_l and out is shape->dtype
+ *    (bf16 or fp32). fp32 inputs are narrowed to bf16 on entry (the tensor
+ *    cores compute in bf16 with fp32 accumulation); d < 128 is zero-padded to
+ *    128 internally.
+ *  - All tensor pointers are DEVICE pointers, 16-byte aligned, owned by the
+ *    caller; except shape->off_host, which is a host pointer. The library
+ *    never allocates, frees or synchronises on the caller's behalf: it
+ *    enqueues kernels on `stream` (a cudaStream_t, NULL = legacy default
+ *    stream) and returns. `workspace` must hold at least
+ *    vdn_workspace_bytes(shape) bytes and stay valid until the work
+ *    completes; calls that share a workspace must be ordered on one stream.
+ *  - Errors: every argument is validated on the host before anything is
+ *    launched, so a call that returns an error has written nothing.
+ *    Return value 0 = VDN_OK, otherwise one of the negative VDN_ERR_* codes.
+ *    VDN_ERR_CUDA reports a launch failure (cudaGetLastError). Device-side
+ *    failures (a bounded wait that expired) are reported by
+ *    vdn_get_device_error() after the caller synchronises.
+ *  - Sizes: 2 <= F <= 4096, 0 <= T, 1 <= H, d in {32, 64, 128},
+ *    block_frames >= 1, lambda > 0, rms_eps >= 0, frame sizes
+ *    off[f+1] - off[f] >= 0, N * H * 128 < 2^31.
+ */
+#ifndef VDN_H_
+#define VDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VDN_OK 0
+#define VDN_ERR_INVALID_ARG (-1)
+#define VDN_ERR_UNSUPPORTED (-2)
+#define VDN_ERR_WORKSPACE_TOO_SMALL (-3)
+#define VDN_ERR_MISALIGNED (-4)
+#define VDN_ERR_CUDA (-5)
+#define VDN_ERR_DEVICE_TIMEOUT (-6)
+#define VDN_ERR_DEVICE (-7)
+
+typedef enum { VDN_BF16 = 0, VDN_F32 = 1 } vdn_dtype_t;
+
+typedef struct vdn_shape {
+  int32_t F;            /* latent frames                                   */
+  int32_t T;            /* text tokens (0 allowed: S_text = 0)             */
+  int32_t H;            /* heads                                           */
+  int32_t d;            /* head dim: 32, 64 or 128                         */
+  int32_t block_frames; /* frames per block; 5 on the pages                */
+  float lambda;         /* VDA ridge weight; 1.0                           */
+  float rms_eps;        /* RMSNorm epsilon; 1e-6                           */
+  int32_t dtype;        /* vdn_dtype_t of the activations                  */
+  const int32_t* off_host; /* [F+1] host copy of frame offsets (off[0]=0)   */
+  const int32_t* off_dev;  /* [F+1] device copy of the same offsets         */
+} vdn_shape_t;
+
+/* Bytes of workspace every entry point below needs for this shape
+ * (the maximum over entry points). Returns 0 if the shape is invalid. */
+size_t vdn_workspace_bytes(const vdn_shape_t* shape);
+
+/* Whole layer: softmax branch, VDA scans, readout, RMSNorm and gated merge.
+ * Writes out [N, H, d] (dtype). rms_w may not be NULL. kt/vt may be NULL iff
+ * T == 0. */
+int vdn_hybrid_attn_fwd(const vdn_shape_t* shape, const void* q, const void* k,
+                        const void* v, const void* kt, const void* vt,
+                        const void* g_s, const void* g_l, const float* rms_w,
+                        void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Linear branch states only. read_states [nb, H, d, d] fp32 (required;
+ * nb = ceil(F / block_frames)) gets R_b. Optional (NULL to skip):
+ * text_state [H, d, d]; fwd_states [F, H, d, d] gets Sfwd[i] for
+ * i = 0..F-2 (entry F-1 is not written); bwd_states [F, H, d, d] gets
+ * Sbwd[j] for j = 1..F-1 (entry 0 is not written). */
+int vdn_vda_scan(const vdn_shape_t* shape, const void* k, const void* v,
+                 const void* kt, const void* vt, float* read_states,
+                 float* text_state, float* fwd_states, float* bwd_states,
+                 void* workspace, size_t ws_bytes, void* stream);
+
+/* Readout and merge only: o_lin = q^T R_b, RMSNorm, sigmoid gates.
+ * read_states [nb, H, d, d] fp32 as written by vdn_vda_scan; o_soft
+ * [N, H, d] bf16 as written by vdn_bsa_fwd. Writes out [N, H, d] (dtype). */
+int vdn_gate_merge(const vdn_shape_t* shape, const void* q,
+                   const float* read_states, const void* o_soft,
+                   const void* g_s, const void* g_l, const float* rms_w,
+                   void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Softmax branch only. Writes o_soft [N, H, d] bf16 and, if lse != NULL,
+ * lse [H, N] fp32 = log(sum_j exp(q.k_j / sqrt(d))) over the allowed keys. */
+int vdn_bsa_fwd(const vdn_shape_t* shape, const void* q, const void* k,
+                const void* v, const void* kt, const void* vt, void* o_soft,
+                float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/* Audit of the block schedule the kernels run: soft_pairs [F, F+1] int64
+ * (device) counts the (query token, key token) pairs the softmax kernel
+ * visits, per (query frame, key frame), with column F counting text keys;
+ * lin_pairs [F, F] int64 (device) counts the pairs folded into the read
+ * states the readout uses. Both are zeroed first. */
+int vdn_pair_audit(const vdn_shape_t* shape, int64_t* soft_pairs,
+                   int64_t* lin_pairs, void* stream);
+
+/* Synchronises the current device, returns VDN_OK or the first device-side
+ * error recorded since the last call (VDN_ERR_DEVICE_TIMEOUT for an expired
+ * bounded wait), and clears it. */
+int vdn_get_device_error(void);
+
+/* Static string for a return code. */
+const char* vdn_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VDN_H_ */

@@ -1,0 +1,145 @@
+"""Host-side checks of the C-ABI boundary: the library loads, exports every
+function include/vdn.h declares, sizes its workspace, and rejects bad
+arguments with the documented error codes before touching the GPU.
+
+Every call here fails host validation, so these tests never launch a kernel
+and never dereference the fake (but aligned) device addresses they pass."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import vdn_synth as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vdn.h")
+
+V = pytest.importorskip("video_diffusion_hybrid_block_b200")
+from video_diffusion_hybrid_block_b200 import binding as B  # noqa: E402
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
+FAKE_MIS = FAKE + 8
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        from video_diffusion_hybrid_block_b200 import build
+        build.build()
+    return B.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("vdn_hybrid_attn_fwd", "vdn_vda_scan", "vdn_gate_merge", "vdn_bsa_fwd",
+              "vdn_pair_audit", "vdn_workspace_bytes", "vdn_get_device_error",
+              "vdn_error_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(B.EXPORTED) == set(declared_functions())
+
+
+def shape(off=None, T=8, H=2, d=128, bf=5, lam=1.0, eps=1e-6, dtype=0):
+    if off is None:
+        off = S.frame_offsets([24] * 10)
+    return V.Shape(off, T, H, d, bf, lam, eps, dtype, device="cpu")
+
+
+def test_workspace_bytes(lib):
+    for name in ("tiny", "pages-scale", "vda-stress"):
+        cfg = S.CONFIGS[name]
+        off = S.frame_offsets(S.frame_sizes(cfg))
+        n = V.vdn_workspace_bytes(shape(off, cfg["T"], cfg["H"], cfg["d"],
+                                        dtype=0 if cfg["dtype"] == "bf16" else 1))
+        N = int(off[-1])
+        assert n >= N * cfg["H"] * 128 * 2  # at least the o_soft buffer
+        assert n % 256 == 0
+    assert V.vdn_workspace_bytes(shape(d=48)) == 0
+    assert V.vdn_workspace_bytes(shape(off=[0, 5])) == 0   # F = 1
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(off=[0, 5]), B.VDN_ERR_INVALID_ARG),                  # F < 2
+    (dict(off=[1, 5, 9]), B.VDN_ERR_INVALID_ARG),               # off[0] != 0
+    (dict(off=[0, 5, 3, 9]), B.VDN_ERR_INVALID_ARG),            # not monotone
+    (dict(d=48), B.VDN_ERR_UNSUPPORTED),
+    (dict(d=256), B.VDN_ERR_UNSUPPORTED),
+    (dict(H=0), B.VDN_ERR_INVALID_ARG),
+    (dict(T=-1), B.VDN_ERR_INVALID_ARG),
+    (dict(bf=0), B.VDN_ERR_INVALID_ARG),
+    (dict(lam=0.0), B.VDN_ERR_INVALID_ARG),
+    (dict(lam=float("nan")), B.VDN_ERR_INVALID_ARG),
+    (dict(eps=-1.0), B.VDN_ERR_INVALID_ARG),
+    (dict(dtype=7), B.VDN_ERR_UNSUPPORTED),
+])
+def test_bad_shapes(lib, kw, code):
+    s = shape(**kw)
+    rc = lib.vdn_hybrid_attn_fwd(s.ref, *([FAKE] * 9), FAKE, 1 << 40, 0)
+    assert rc == code
+    rc = lib.vdn_bsa_fwd(s.ref, *([FAKE] * 7), FAKE, 1 << 40, 0)
+    assert rc == code
+    rc = lib.vdn_vda_scan(s.ref, *([FAKE] * 8), FAKE, 1 << 40, 0)
+    assert rc == code
+
+
+def test_null_shape(lib):
+    assert lib.vdn_hybrid_attn_fwd(None, *([FAKE] * 9), FAKE, 1 << 40, 0) == B.VDN_ERR_INVALID_ARG
+    assert lib.vdn_workspace_bytes(None) == 0
+
+
+def test_null_and_misaligned_pointers(lib):
+    s = shape()
+    ptrs = [FAKE] * 9
+    for i in range(9):
+        p = list(ptrs)
+        p[i] = 0
+        assert lib.vdn_hybrid_attn_fwd(s.ref, *p, FAKE, 1 << 40, 0) == B.VDN_ERR_INVALID_ARG, i
+        p[i] = FAKE_MIS
+        assert lib.vdn_hybrid_attn_fwd(s.ref, *p, FAKE, 1 << 40, 0) == B.VDN_ERR_MISALIGNED, i
+    # text pointers may be NULL when T == 0, but then the workspace check fails
+    s0 = shape(T=0)
+    p = [FAKE] * 9
+    p[3] = p[4] = 0
+    assert lib.vdn_hybrid_attn_fwd(s0.ref, *p, FAKE, 16, 0) == B.VDN_ERR_WORKSPACE_TOO_SMALL
+    assert lib.vdn_pair_audit(s.ref, None, FAKE, 0) == B.VDN_ERR_INVALID_ARG
+
+
+def test_workspace_too_small_and_misaligned(lib):
+    s = shape()
+    need = V.vdn_workspace_bytes(s)
+    assert lib.vdn_hybrid_attn_fwd(s.ref, *([FAKE] * 9), FAKE, need - 1, 0) == \
+        B.VDN_ERR_WORKSPACE_TOO_SMALL
+    assert lib.vdn_hybrid_attn_fwd(s.ref, *([FAKE] * 9), None, need, 0) == \
+        B.VDN_ERR_WORKSPACE_TOO_SMALL
+    assert lib.vdn_hybrid_attn_fwd(s.ref, *([FAKE] * 9), FAKE_MIS, need, 0) == \
+        B.VDN_ERR_MISALIGNED
+    assert lib.vdn_vda_scan(s.ref, *([FAKE] * 8), FAKE, need - 1, 0) == \
+        B.VDN_ERR_WORKSPACE_TOO_SMALL
+    assert lib.vdn_gate_merge(s.ref, *([FAKE] * 7), FAKE, need - 1, 0) == \
+        B.VDN_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_error_strings(lib):
+    for code in range(-7, 1):
+        assert len(B.vdn_error_string(code)) > 0
+    assert B.vdn_error_string(-99) == "unknown error"
+
+
+def test_binding_raises_on_error(lib):
+    s = shape(d=48)
+    with pytest.raises(B.VdnError) as e:
+        V.vdn_hybrid_attn_fwd(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              stream=0, ws_bytes=1 << 40)
+    assert e.value.code == B.VDN_ERR_UNSUPPORTED

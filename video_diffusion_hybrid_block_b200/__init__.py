@@ -1,0 +1,10 @@
+"""B200 (sm_100a) forward pass of VideoDeltaNet's hybrid attention layer.
+
+The compute lives in libvdn.so (C ABI, include/vdn.h); ``binding`` marshals
+torch tensors into it.
+"""
+from .binding import (  # noqa: F401
+    EXPORTED, LIB_PATH, VDN_BF16, VDN_F32, Shape, VdnError, alloc_workspace, load_library,
+    vdn_bsa_fwd, vdn_error_string, vdn_gate_merge, vdn_get_device_error, vdn_hybrid_attn_fwd,
+    vdn_pair_audit, vdn_vda_scan, vdn_workspace_bytes,
+)

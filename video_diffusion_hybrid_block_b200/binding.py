@@ -1,0 +1,204 @@
+"""ctypes binding of the C ABI declared in include/vdn.h.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels
+of libvdn.so. Tensors are torch CUDA tensors (PyTorch supplies device memory
+and streams); the functions pass their data pointers and the current stream.
+There is no fallback: if libvdn.so is missing this module raises on import
+of the library.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+VDN_OK = 0
+VDN_ERR_INVALID_ARG = -1
+VDN_ERR_UNSUPPORTED = -2
+VDN_ERR_WORKSPACE_TOO_SMALL = -3
+VDN_ERR_MISALIGNED = -4
+VDN_ERR_CUDA = -5
+VDN_ERR_DEVICE_TIMEOUT = -6
+VDN_ERR_DEVICE = -7
+
+VDN_BF16 = 0
+VDN_F32 = 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdn.so")
+
+
+class VdnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {vdn_error_string(code)} ({code})")
+
+
+class vdn_shape_t(ctypes.Structure):
+    _fields_ = [
+        ("F", ctypes.c_int32),
+        ("T", ctypes.c_int32),
+        ("H", ctypes.c_int32),
+        ("d", ctypes.c_int32),
+        ("block_frames", ctypes.c_int32),
+        ("lambda_", ctypes.c_float),
+        ("rms_eps", ctypes.c_float),
+        ("dtype", ctypes.c_int32),
+        ("off_host", ctypes.POINTER(ctypes.c_int32)),
+        ("off_dev", ctypes.POINTER(ctypes.c_int32)),
+    ]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+_SIGS = {
+    "vdn_workspace_bytes": (_SZ, [ctypes.POINTER(vdn_shape_t)]),
+    "vdn_hybrid_attn_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 9 + [_P, _SZ, _P]),
+    "vdn_vda_scan": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 8 + [_P, _SZ, _P]),
+    "vdn_gate_merge": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
+    "vdn_bsa_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
+    "vdn_pair_audit": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t), _P, _P, _P]),
+    "vdn_get_device_error": (ctypes.c_int, []),
+    "vdn_error_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+EXPORTED = tuple(_SIGS)
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libvdn.so (raises OSError if it is missing: no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise OSError(f"{path} is not built; run `python -m video_diffusion_hybrid_block_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def vdn_error_string(code: int) -> str:
+    try:
+        return load_library().vdn_error_string(int(code)).decode()
+    except OSError:
+        return f"error {code}"
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the C ABI must be contiguous")
+    return t.data_ptr()
+
+
+def _nbytes(workspace, ws_bytes) -> int:
+    if ws_bytes is not None:
+        return int(ws_bytes)
+    if workspace is None or isinstance(workspace, int):
+        return 0
+    return workspace.numel() * workspace.element_size()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class Shape:
+    """Owns a vdn_shape_t plus the host/device frame-offset arrays it points to."""
+
+    def __init__(self, off, T: int, H: int, d: int, block_frames: int = 5,
+                 lam: float = 1.0, rms_eps: float = 1e-6, dtype: int = VDN_BF16,
+                 device=None):
+        self.off_host = torch.as_tensor(off, dtype=torch.int32).contiguous().cpu()
+        # device copy read by the kernels; "cpu" only for host-side argument checks
+        self.off_dev = self.off_host.clone() if str(device) == "cpu" else self.off_host.to(device or "cuda")
+        self.F = len(self.off_host) - 1
+        self.N = int(self.off_host[-1])
+        self.T, self.H, self.d = int(T), int(H), int(d)
+        self.block_frames = int(block_frames)
+        self.nb = -(-self.F // self.block_frames) if self.block_frames > 0 else 0
+        self.c = vdn_shape_t(
+            self.F, self.T, self.H, self.d, self.block_frames, float(lam),
+            float(rms_eps), int(dtype),
+            ctypes.cast(self.off_host.data_ptr(), ctypes.POINTER(ctypes.c_int32)),
+            ctypes.cast(self.off_dev.data_ptr(), ctypes.POINTER(ctypes.c_int32)))
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def _check(rc: int, where: str):
+    if rc != VDN_OK:
+        raise VdnError(rc, where)
+
+
+def vdn_workspace_bytes(shape: Shape) -> int:
+    return int(load_library().vdn_workspace_bytes(shape.ref))
+
+
+def vdn_hybrid_attn_fwd(shape: Shape, q, k, v, kt, vt, g_s, g_l, rms_w, out, workspace,
+                        stream=None, ws_bytes=None):
+    rc = load_library().vdn_hybrid_attn_fwd(
+        shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(g_s), _ptr(g_l),
+        _ptr(rms_w), _ptr(out), _ptr(workspace), _nbytes(workspace, ws_bytes),
+        _stream(stream))
+    _check(rc, "vdn_hybrid_attn_fwd")
+    return out
+
+
+def vdn_vda_scan(shape: Shape, k, v, kt, vt, read_states, text_state, fwd_states, bwd_states,
+                 workspace, stream=None, ws_bytes=None):
+    rc = load_library().vdn_vda_scan(
+        shape.ref, _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(read_states), _ptr(text_state),
+        _ptr(fwd_states), _ptr(bwd_states), _ptr(workspace),
+        _nbytes(workspace, ws_bytes), _stream(stream))
+    _check(rc, "vdn_vda_scan")
+    return read_states
+
+
+def vdn_gate_merge(shape: Shape, q, read_states, o_soft, g_s, g_l, rms_w, out, workspace,
+                   stream=None, ws_bytes=None):
+    rc = load_library().vdn_gate_merge(
+        shape.ref, _ptr(q), _ptr(read_states), _ptr(o_soft), _ptr(g_s), _ptr(g_l), _ptr(rms_w),
+        _ptr(out), _ptr(workspace), _nbytes(workspace, ws_bytes),
+        _stream(stream))
+    _check(rc, "vdn_gate_merge")
+    return out
+
+
+def vdn_bsa_fwd(shape: Shape, q, k, v, kt, vt, o_soft, lse, workspace, stream=None,
+                ws_bytes=None):
+    rc = load_library().vdn_bsa_fwd(
+        shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(o_soft), _ptr(lse),
+        _ptr(workspace), _nbytes(workspace, ws_bytes), _stream(stream))
+    _check(rc, "vdn_bsa_fwd")
+    return o_soft
+
+
+def vdn_pair_audit(shape: Shape, soft_pairs, lin_pairs, stream=None):
+    rc = load_library().vdn_pair_audit(shape.ref, _ptr(soft_pairs), _ptr(lin_pairs),
+                                       _stream(stream))
+    _check(rc, "vdn_pair_audit")
+    return soft_pairs, lin_pairs
+
+
+def vdn_get_device_error() -> int:
+    return int(load_library().vdn_get_device_error())
+
+
+def alloc_workspace(shape: Shape, device=None) -> torch.Tensor:
+    n = vdn_workspace_bytes(shape)
+    if n == 0:
+        raise VdnError(VDN_ERR_INVALID_ARG, "vdn_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")

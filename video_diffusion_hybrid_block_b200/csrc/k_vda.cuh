@@ -1,0 +1,454 @@
+// Video Delta Attention (linear branch): per-frame Grams, per-frame SPD
+// inverses and the two text-initialised state scans.
+//
+// VDA replaces the token-by-token delta rule with one joint solve per frame:
+// the normal equations of all spatial tokens of the frame determine the new
+// state; the text writes the state once at initialisation; the branch sums
+// the context before and after the current window
+// [nav.superapi.store page, Technical Principles, Video Delta Attention and
+// Text Dual-Branch Injection; "VDN-MiniMax-H3" (openi.cn), 技术原理].
+// Reading implemented: k_hat = k / max(||k||, 1e-12),
+//   M_f = lambda I + K_f^T K_f, C_f = K_f^T V_f,
+//   S_f = M_f^-1 (lambda S_prev + C_f), S_text = M_t^-1 C_t.
+//
+// k_vda_gram_inv: one CTA per (matrix m, head): m = 0 is the text, m = f is
+//   latent frame f (1 <= f <= F-2; anchors 0 and F-1 are never scanned).
+//   Streams the frame's k, v rows in 64-token tiles (TMA, 2 stages),
+//   L2-normalises k rows in shared memory, accumulates [G | C] = K^T [K | V]
+//   as one M=128 x N=256 bf16 tcgen05 contraction into TMEM, writes C (fp32)
+//   and then inverts M = lambda I + G in registers with a Gauss-Jordan sweep
+//   (no pivoting: M is symmetric positive definite with eigenvalues
+//   >= lambda) and writes W = M^-1 (fp32).
+// k_vda_scan: one CTA per (direction, head). Step 0 applies the text
+//   (S = W_t C_t), then one step per frame: X = lambda S + C_f,
+//   S = W_f X as a tf32 tcgen05 contraction (W via TMA, X written
+//   transposed by the threads, D in TMEM). States a block reads go to
+//   Rpart[dir][b]; optional per-frame / text outputs are written too.
+#pragma once
+
+#include "layer_plan.cuh"
+#include "sm100_ptx.cuh"
+
+namespace vdn {
+
+// ------------------------------------------------------------ Gram + inverse
+
+constexpr int kGramThreads = 256;
+constexpr int kGramTok = 64;                // tokens per tile
+constexpr uint32_t kGramStage = 4 * 8192;  // k chunk0, k chunk1, v chunk0, v chunk1
+// 2 stages (64 KB); the request is padded so at most two CTAs share an SM
+// (two x 256 TMEM columns).
+constexpr uint32_t kGramSmemBytes = 100 * 1024;
+
+struct GramParams {
+  const int32_t* off;  // [F+1] device
+  int F, T, H;
+  float lambda;
+  float* Cmat;  // [F-1][H][128][128]
+  float* Wmat;  // [F-1][H][128][128]
+};
+
+__global__ void __launch_bounds__(kGramThreads, 2)
+    k_vda_gram_inv(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                   const __grid_constant__ CUtensorMap tkt, const __grid_constant__ CUtensorMap tvt,
+                   const GramParams p) {
+  const int m = blockIdx.x, h = blockIdx.y;
+  const bool text = (m == 0);
+  const int r0 = text ? 0 : p.off[m];
+  const int r1 = text ? p.T : p.off[m + 1];
+  const int nrows = r1 - r0;
+  const int ntiles = (nrows + kGramTok - 1) / kGramTok;
+  const CUtensorMap* mk = text ? &tkt : &tk;
+  const CUtensorMap* mv = text ? &tvt : &tv;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_full[2], bar_empty[2], bar_done;
+  __shared__ uint32_t tmem_slot;
+  __shared__ float rowbuf[2][128], colbuf[2][128];
+  __shared__ int abort_flag;
+
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t full[2] = {smem_u32(&bar_full[0]), smem_u32(&bar_full[1])};
+  const uint32_t empty[2] = {smem_u32(&bar_empty[0]), smem_u32(&bar_empty[1])};
+  const uint32_t done = smem_u32(&bar_done);
+  volatile int* abort_v = &abort_flag;
+
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(full[i], 1);
+      mbar_init(empty[i], 1);
+    }
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  auto load_tile = [&](int i, int st) {
+    const uint32_t dst = base + (uint32_t)st * kGramStage;
+    const int row = r0 + i * kGramTok;
+    mbar_arrive_expect_tx(full[st], kGramStage);
+    tma_load_3d(dst, mk, full[st], 0, h, row);
+    tma_load_3d(dst + 8192, mk, full[st], 64, h, row);
+    tma_load_3d(dst + 16384, mv, full[st], 0, h, row);
+    tma_load_3d(dst + 24576, mv, full[st], 64, h, row);
+  };
+  if (tid == 0) {
+    for (int i = 0; i < imin(2, ntiles); ++i) load_tile(i, i);
+  }
+
+  const uint32_t idG = idesc_bf16(128, 256, true, true);
+  bool ok = true;
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i & 1;
+    const uint32_t ph = (i >> 1) & 1;
+    if (*abort_v || !mbar_wait(full[st], ph)) { ok = false; *abort_v = 1; }
+    __syncthreads();
+    if (*abort_v) { ok = false; break; }
+    // L2-normalise k rows (zero rows beyond the frame, and their v rows)
+    const uint32_t stage = base + (uint32_t)st * kGramStage;
+    const int row = tid >> 2, quarter = tid & 3;
+    const uint32_t chunk = (uint32_t)(quarter >> 1);
+    const uint32_t u0 = (uint32_t)((quarter & 1) * 4);
+    uint4 kv[4];
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      kv[u] = ld_shared_v4(stage + chunk * 8192 + sw128_off((uint32_t)row, u0 + u));
+      const uint32_t w4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = bf_lo(w4[e]), b = bf_hi(w4[e]);
+        ss = fmaf(a, a, fmaf(b, b, ss));
+      }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    const bool valid = (i * kGramTok + row) < nrows;
+    const float sc = valid ? 1.f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t w4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+      uint32_t o4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o4[e] = pack_bf16x2(bf_lo(w4[e]) * sc, bf_hi(w4[e]) * sc);
+      st_shared_v4(stage + chunk * 8192 + sw128_off((uint32_t)row, u0 + u), o4[0], o4[1], o4[2],
+                   o4[3]);
+      if (!valid)
+        st_shared_v4(stage + 16384 + chunk * 8192 + sw128_off((uint32_t)row, u0 + u), 0u, 0u, 0u,
+                     0u);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint64_t d = sdesc_sw128(stage + (uint32_t)(s * 2048), 8192, 1024);
+        umma_bf16_ss(tmem, d, d, idG, (i > 0 || s > 0) ? 1u : 0u);
+      }
+      umma_commit(empty[st]);
+      if (i == ntiles - 1) umma_commit(done);
+      if (i + 2 < ntiles) {
+        if (!mbar_wait(empty[st], ph)) {
+          *abort_v = 1;
+        } else {
+          load_tile(i + 2, st);
+        }
+      }
+    }
+  }
+  if (ok && ntiles > 0 && !mbar_wait(done, 0)) ok = false;
+  if (!ok) *abort_v = 1;
+  tc_fence_after();
+  __syncthreads();
+
+  // TMEM -> C (global, fp32) and G (shared, fp32, 16-byte units XOR-swizzled)
+  const uint32_t gs = base;  // reuses the (now idle) staging buffers: 64 KB
+  {
+    const int wq = warp & 3;
+    const int i = wq * 32 + lane;
+    float* cdst = p.Cmat + (((int64_t)m * p.H + h) * 128 + i) * 128;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      if (ntiles > 0) {
+        tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + (warp < 4 ? 0u : 128u) + (uint32_t)(c * 32), r);
+        tmem_ld_wait(r);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = 0u;
+      }
+#pragma unroll
+      for (int uu = 0; uu < 8; ++uu) {
+        const int u = c * 8 + uu;
+        if (warp >= 4)
+          reinterpret_cast<uint4*>(cdst)[u] =
+              make_uint4(r[4 * uu], r[4 * uu + 1], r[4 * uu + 2], r[4 * uu + 3]);
+        else
+          st_shared_v4(gs + (uint32_t)i * 512u + (((uint32_t)u ^ (uint32_t)(i & 31)) << 4),
+                       r[4 * uu], r[4 * uu + 1], r[4 * uu + 2], r[4 * uu + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+
+  // Gauss-Jordan inverse of M = lambda I + G, 8x8 register tile per thread.
+  const int ty = tid >> 4, tx = tid & 15;
+  float a[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t R = (uint32_t)(8 * ty + i);
+#pragma unroll
+    for (int hlf = 0; hlf < 2; ++hlf) {
+      const uint4 v = ld_shared_v4(gs + R * 512u + ((((uint32_t)(2 * tx + hlf)) ^ (R & 31u)) << 4));
+      a[i][4 * hlf + 0] = __uint_as_float(v.x);
+      a[i][4 * hlf + 1] = __uint_as_float(v.y);
+      a[i][4 * hlf + 2] = __uint_as_float(v.z);
+      a[i][4 * hlf + 3] = __uint_as_float(v.w);
+    }
+  }
+  if (ty == tx) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i][i] += p.lambda;
+  }
+  for (int kb8 = 0; kb8 < 16; ++kb8) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int k = kb8 * 8 + kk;
+      const int buf = k & 1;
+      if (ty == kb8) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rowbuf[buf][8 * tx + j] = a[kk][j];
+      }
+      if (tx == kb8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) colbuf[buf][8 * ty + i] = a[i][kk];
+      }
+      __syncthreads();
+      const float ip = 1.f / rowbuf[buf][k];
+      float rj[8], ci[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) rj[j] = rowbuf[buf][8 * tx + j] * ip;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ci[i] = colbuf[buf][8 * ty + i];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[i][j] = fmaf(-ci[i], rj[j], a[i][j]);
+      if (ty == kb8) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[kk][j] = rj[j];
+      }
+      if (tx == kb8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i][kk] = -ci[i] * ip;
+      }
+      if (ty == kb8 && tx == kb8) a[kk][kk] = ip;
+    }
+  }
+  float* wdst = p.Wmat + ((int64_t)m * p.H + h) * 128 * 128;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float4* rowp = reinterpret_cast<float4*>(wdst + (int64_t)(8 * ty + i) * 128 + 8 * tx);
+    rowp[0] = make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
+    rowp[1] = make_float4(a[i][4], a[i][5], a[i][6], a[i][7]);
+  }
+}
+
+// --------------------------------------------------------------- scans ----
+
+constexpr int kScanThreads = 128;
+constexpr uint32_t kScanSmemW = 0;          // 2 stages x 64 KB
+constexpr uint32_t kScanSmemX = 2 * 65536;  // X^T, 64 KB
+constexpr uint32_t kScanSmemBytes = 3 * 65536 + 1024;
+
+struct ScanParams {
+  const float* Cmat;  // [F-1][H][128][128]
+  int F, H, bf, nb;
+  float lambda;
+  float* Rpart;       // [2][nb][H][128][128]
+  float* text_out;    // optional [H][d][d]
+  float* fwd_out;     // optional [F][H][d][d]
+  float* bwd_out;     // optional [F][H][d][d]
+  int d_out;
+};
+
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(__float_as_uint(v)) : "memory");
+}
+
+__global__ void __launch_bounds__(kScanThreads, 1)
+    k_vda_scan(const __grid_constant__ CUtensorMap tw, const ScanParams p) {
+  const int dir = blockIdx.x, h = blockIdx.y;
+  const int F = p.F;
+  const int nsteps = F - 1;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t bar_w[2], bar_mma;
+  __shared__ uint32_t tmem_slot;
+
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sW[2] = {base + kScanSmemW, base + kScanSmemW + 65536};
+  const uint32_t sX = base + kScanSmemX;
+  const int i = threadIdx.x, warp = i >> 5;
+  const uint32_t wfull[2] = {smem_u32(&bar_w[0]), smem_u32(&bar_w[1])};
+  const uint32_t mma_bar = smem_u32(&bar_mma);
+
+  if (i == 0) {
+    mbar_init(wfull[0], 1);
+    mbar_init(wfull[1], 1);
+    mbar_init(mma_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+
+  auto mat_of = [&](int s) -> int { return (s == 0) ? 0 : (dir == 0 ? s : F - 1 - s); };
+  auto idx_of = [&](int s) -> int { return dir == 0 ? s : (s == 0 ? F - 1 : F - 1 - s); };
+  auto load_w = [&](int s, int st) {
+    const int row = (mat_of(s) * p.H + h) * 128;
+    mbar_arrive_expect_tx(wfull[st], 65536);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tma_load_2d(sW[st] + (uint32_t)(c * 16384), &tw, wfull[st], c * 32, row);
+  };
+  if (i == 0) {
+    tma_prefetch_desc(&tw);
+    load_w(0, 0);
+    if (nsteps > 1) load_w(1, 1);
+  }
+
+  float creg[128];
+  {
+    const float4* src = reinterpret_cast<const float4*>(
+        p.Cmat + (((int64_t)mat_of(0) * p.H + h) * 128 + i) * 128);
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const float4 v = __ldg(src + u);
+      creg[4 * u] = v.x; creg[4 * u + 1] = v.y; creg[4 * u + 2] = v.z; creg[4 * u + 3] = v.w;
+    }
+  }
+  const uint32_t xcol = sX + (uint32_t)(i >> 5) * 16384u;  // k chunk of this thread's column
+  const uint32_t xu = (uint32_t)((i & 31) >> 2), xb = (uint32_t)((i & 3) * 4);
+  const uint32_t idW = idesc_tf32(128, 128, false, false);
+  bool ok = true;
+
+  for (int s = 0; s < nsteps && ok; ++s) {
+    // X = lambda * S_prev + C, stored transposed (row n, column i) in 128B-swizzled K-major form
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t sv[32];
+      if (s > 0) {
+        tmem_ld32(tmem + lane_base + (uint32_t)(c * 32), sv);
+        tmem_ld_wait(sv);
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) sv[jj] = 0u;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        const int n = c * 32 + jj;
+        const float x = fmaf(p.lambda, __uint_as_float(sv[jj]), creg[n]);
+        st_shared_f32(xcol + sw128_off((uint32_t)n, xu) + xb, x);
+      }
+    }
+    if (s + 1 < nsteps) {
+      const float4* src = reinterpret_cast<const float4*>(
+          p.Cmat + (((int64_t)mat_of(s + 1) * p.H + h) * 128 + i) * 128);
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const float4 v = __ldg(src + u);
+        creg[4 * u] = v.x; creg[4 * u + 1] = v.y; creg[4 * u + 2] = v.z; creg[4 * u + 3] = v.w;
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_barrier_sync(1, kScanThreads);
+    if (i == 0) {
+      const int st = s & 1;
+      if (!mbar_wait(wfull[st], (uint32_t)((s >> 1) & 1))) {
+        ok = false;
+      } else {
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint32_t ko = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32);
+          umma_tf32_ss(tmem, sdesc_sw128(sW[st] + ko, 16, 1024), sdesc_sw128(sX + ko, 16, 1024),
+                       idW, k > 0 ? 1u : 0u);
+        }
+        umma_commit(mma_bar);
+      }
+    }
+    if (!mbar_wait(mma_bar, (uint32_t)(s & 1))) { ok = false; break; }
+    tc_fence_after();
+    if (i == 0 && s + 2 < nsteps) load_w(s + 2, s & 1);
+
+    // outputs of this state
+    const int idx = idx_of(s);
+    bool want = (dir == 0 && p.fwd_out != nullptr) || (dir == 1 && p.bwd_out != nullptr) ||
+                (s == 0 && dir == 0 && p.text_out != nullptr);
+    for (int b = 0; b < p.nb && !want; ++b) {
+      int i_f, i_b;
+      block_read_indices(b, F, p.bf, i_f, i_b);
+      want = (dir == 0 ? i_f : i_b) == idx;
+    }
+    if (want) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(c * 32), sv);
+        tmem_ld_wait(sv);
+        for (int b = 0; b < p.nb; ++b) {
+          int i_f, i_b;
+          block_read_indices(b, F, p.bf, i_f, i_b);
+          if ((dir == 0 ? i_f : i_b) != idx) continue;
+          float* dst = p.Rpart + ((((int64_t)dir * p.nb + b) * p.H + h) * 128 + i) * 128 + c * 32;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            reinterpret_cast<uint4*>(dst)[u] =
+                make_uint4(sv[4 * u], sv[4 * u + 1], sv[4 * u + 2], sv[4 * u + 3]);
+        }
+        if (i < p.d_out) {
+          float* outs[3] = {nullptr, nullptr, nullptr};
+          if (dir == 0 && p.fwd_out) outs[0] = p.fwd_out + (((int64_t)idx * p.H + h) * p.d_out + i) * p.d_out;
+          if (dir == 1 && p.bwd_out) outs[1] = p.bwd_out + (((int64_t)idx * p.H + h) * p.d_out + i) * p.d_out;
+          if (s == 0 && dir == 0 && p.text_out) outs[2] = p.text_out + ((int64_t)h * p.d_out + i) * p.d_out;
+#pragma unroll
+          for (int o = 0; o < 3; ++o) {
+            if (outs[o] == nullptr) continue;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+              if (c * 32 + jj < p.d_out) outs[o][c * 32 + jj] = __uint_as_float(sv[jj]);
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+}  // namespace vdn

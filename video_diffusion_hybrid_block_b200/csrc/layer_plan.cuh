@@ -1,0 +1,108 @@
+// Integer structure of the hybrid layer, shared by host and device code:
+// frame blocks, softmax windows with boundary anchors, key segments of a
+// query block, the scan states a block reads.
+//
+// Blocks of `bf` consecutive latent frames; block b's softmax window is
+// blocks b-1..b+1 (clipped), plus frames 0 and F-1 as boundary anchors, plus
+// every text token ["VDN-MiniMax-H3" (openi.cn), 技术原理：局部精确、远程压缩;
+// nav.superapi.store page, Technical Principles, Local Softmax Branch and
+// Text Dual-Branch Injection]. The linear branch of block b reads the forward
+// state just before its window and the backward state just after it, both
+// excluding window frames and anchors [openi.cn page, same section].
+#pragma once
+
+#include <stdint.h>
+
+namespace vdn {
+
+constexpr int kTile = 128;   // query rows / key rows per softmax tile
+constexpr int kDPad = 128;   // head dim the kernels run at (smaller d is zero-padded)
+constexpr int kMaxSegs = 4;  // text + at most three video ranges
+
+__host__ __device__ inline int imin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ inline int imax(int a, int b) { return a > b ? a : b; }
+
+__host__ __device__ inline int num_blocks(int F, int bf) { return (F + bf - 1) / bf; }
+
+// First and last frame of block b's window (blocks b-1, b, b+1, clipped).
+__host__ __device__ inline void block_window(int b, int F, int bf, int& w0, int& w1) {
+  w0 = bf * imax(b - 1, 0);
+  w1 = imin(bf * (b + 2), F) - 1;
+}
+
+// Scan-state indices block b reads: forward state after frame w0-1 (index 0
+// is the text-initialised state) and backward state after frame w1+1 (index
+// F-1 is the text-initialised state).
+__host__ __device__ inline void block_read_indices(int b, int F, int bf, int& i_fwd,
+                                                   int& i_bwd) {
+  int w0, w1;
+  block_window(b, F, bf, w0, w1);
+  i_fwd = imax(w0 - 1, 0);
+  i_bwd = imin(w1 + 1, F - 1);
+}
+
+// Query rows of block b: [q0, q1).
+__host__ __device__ inline void block_rows(const int32_t* off, int F, int bf, int b, int& q0,
+                                           int& q1) {
+  q0 = off[bf * b];
+  q1 = off[imin(bf * b + bf, F)];
+}
+
+// Key segments of block b in visiting order: text first, then the video
+// frame ranges {0}, [w0, w1], {F-1} merged where they touch.
+struct KeySegs {
+  int n;
+  int src[kMaxSegs];    // 0 = video k/v rows, 1 = text kt/vt rows
+  int start[kMaxSegs];  // first row in its source
+  int len[kMaxSegs];    // rows
+  int first_tile[kMaxSegs + 1];
+};
+
+__host__ __device__ inline void segs_push(KeySegs& s, int src, int a, int e) {
+  if (e > a) {
+    s.src[s.n] = src;
+    s.start[s.n] = a;
+    s.len[s.n] = e - a;
+    s.first_tile[s.n + 1] = s.first_tile[s.n] + (e - a + kTile - 1) / kTile;
+    s.n++;
+  }
+}
+
+__host__ __device__ inline KeySegs key_segments(const int32_t* off, int F, int bf, int T,
+                                                int b) {
+  KeySegs s;
+  s.n = 0;
+  s.first_tile[0] = 0;
+  segs_push(s, 1, 0, T);
+  int w0, w1;
+  block_window(b, F, bf, w0, w1);
+  // frame ranges, inclusive, in increasing order
+  int ra[3] = {0, w0, F - 1};
+  int rb[3] = {0, w1, F - 1};
+  int ca = ra[0], cb = rb[0];
+  for (int i = 1; i < 3; ++i) {
+    if (ra[i] <= cb + 1) {
+      cb = imax(cb, rb[i]);
+    } else {
+      segs_push(s, 0, off[ca], off[cb + 1]);
+      ca = ra[i];
+      cb = rb[i];
+    }
+  }
+  segs_push(s, 0, off[ca], off[cb + 1]);
+  return s;
+}
+
+__host__ __device__ inline int segs_tiles(const KeySegs& s) { return s.first_tile[s.n]; }
+
+// Key tile j of the list: source, first row, number of valid rows (1..128).
+__host__ __device__ inline void segs_tile(const KeySegs& s, int j, int& src, int& row0,
+                                          int& valid) {
+  int i = 0;
+  while (i + 1 < s.n && j >= s.first_tile[i + 1]) ++i;
+  src = s.src[i];
+  row0 = s.start[i] + (j - s.first_tile[i]) * kTile;
+  valid = imin(kTile, s.start[i] + s.len[i] - row0);
+}
+
+}  // namespace vdn

@@ -1,0 +1,479 @@
+// C ABI of the hybrid attention layer (declared in include/vdn.h).
+// Host side only: argument validation, workspace carving, TMA descriptor
+// encoding and kernel launches on the caller's stream. Single translation
+// unit (the kernels are header-only), so one device error word serves all
+// kernels.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <initializer_list>
+
+#include "../../include/vdn.h"
+#include "k_audit.cuh"
+#include "k_bsa_fwd.cuh"
+#include "k_merge.cuh"
+#include "k_prepare.cuh"
+#include "k_vda.cuh"
+#include "layer_plan.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+using namespace vdn;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows, H, 128] bf16 viewed as a 3-D tensor {128, H, rows}; box {64, 1, box_rows}.
+bool map_act(CUtensorMap* m, const void* ptr, int64_t rows, int H, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kDPad, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)kDPad * 2, (cuuint64_t)H * kDPad * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, 128] fp32 as a 2-D tensor; box {32, 128}.
+bool map_mat(CUtensorMap* m, const void* ptr, int64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)128, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)128 * 4};
+  cuuint32_t box[2] = {32, 128};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+
+__global__ void k_sum_states(const float* a, const float* b, float* out, int64_t n, int d) {
+  // out[(bh, i, j)] = a[(bh, i, j)] + b[(bh, i, j)] with a, b padded to 128 x 128
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n) return;
+  const int64_t bh = t / ((int64_t)d * d);
+  const int r = (int)((t / d) % d), c = (int)(t % d);
+  const int64_t src = (bh * 128 + r) * 128 + c;
+  out[t] = a[src] + b[src];
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Plan {
+  int F, T, H, d, bf, nb, N;
+  float lambda, eps;
+  int dtype;
+  int max_qtiles;
+  bool staged;  // inputs are narrowed / padded into the workspace
+  size_t o_q, o_k, o_v, o_kt, o_vt, o_osoft, o_C, o_W, o_R, total;
+  const int32_t* off_dev;
+};
+
+int make_plan(const vdn_shape_t* s, Plan* P) {
+  if (s == nullptr) return VDN_ERR_INVALID_ARG;
+  if (s->F < 2 || s->F > 4096 || s->T < 0 || s->H < 1 || s->block_frames < 1)
+    return VDN_ERR_INVALID_ARG;
+  if (!(s->d == 32 || s->d == 64 || s->d == 128)) return VDN_ERR_UNSUPPORTED;
+  if (!(s->lambda > 0.f) || !std::isfinite(s->lambda) || !(s->rms_eps >= 0.f) ||
+      !std::isfinite(s->rms_eps))
+    return VDN_ERR_INVALID_ARG;
+  if (s->dtype != VDN_BF16 && s->dtype != VDN_F32) return VDN_ERR_UNSUPPORTED;
+  if (s->off_host == nullptr || s->off_dev == nullptr) return VDN_ERR_INVALID_ARG;
+  if (s->off_host[0] != 0) return VDN_ERR_INVALID_ARG;
+  for (int f = 0; f < s->F; ++f)
+    if (s->off_host[f + 1] < s->off_host[f]) return VDN_ERR_INVALID_ARG;
+  const int64_t N = s->off_host[s->F];
+  if (N * (int64_t)s->H * kDPad >= (int64_t(1) << 31)) return VDN_ERR_UNSUPPORTED;
+  if ((int64_t)s->T * s->H * kDPad >= (int64_t(1) << 31)) return VDN_ERR_UNSUPPORTED;
+  if ((int64_t)(s->F - 1) * s->H * 128 >= (int64_t(1) << 31)) return VDN_ERR_UNSUPPORTED;
+  P->F = s->F;
+  P->T = s->T;
+  P->H = s->H;
+  P->d = s->d;
+  P->bf = s->block_frames;
+  P->nb = num_blocks(s->F, s->block_frames);
+  P->N = (int)N;
+  P->lambda = s->lambda;
+  P->eps = s->rms_eps;
+  P->dtype = s->dtype;
+  P->off_dev = s->off_dev;
+  P->max_qtiles = 0;
+  for (int b = 0; b < P->nb; ++b) {
+    int q0, q1;
+    block_rows(s->off_host, P->F, P->bf, b, q0, q1);
+    P->max_qtiles = imax(P->max_qtiles, (q1 - q0 + kTile - 1) / kTile);
+  }
+  P->staged = (s->dtype != VDN_BF16) || (s->d != kDPad);
+  const size_t act = (size_t)N * P->H * kDPad * 2;
+  const size_t txt = (size_t)P->T * P->H * kDPad * 2;
+  const size_t mat = (size_t)(P->F - 1) * P->H * 128 * 128 * 4;
+  size_t o = 0;
+  P->o_q = o; o += P->staged ? align256(act) : 0;
+  P->o_k = o; o += P->staged ? align256(act) : 0;
+  P->o_v = o; o += P->staged ? align256(act) : 0;
+  P->o_kt = o; o += P->staged ? align256(txt) : 0;
+  P->o_vt = o; o += P->staged ? align256(txt) : 0;
+  P->o_osoft = o; o += align256(act);
+  P->o_C = o; o += align256(mat);
+  P->o_W = o; o += align256(mat);
+  P->o_R = o; o += align256((size_t)2 * P->nb * P->H * 128 * 128 * 4);
+  P->total = o;
+  return VDN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Kernel attribute set-up, once per device.
+bool set_smem_attrs() {
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (done[dev]) return true;
+  bool ok = cudaFuncSetAttribute(k_bsa_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kBsaSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_vda_gram_inv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kGramSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_vda_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kScanSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_readout_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kMergeSmemBytes) == cudaSuccess;
+  done[dev] = ok;
+  return ok;
+}
+
+// bf16 [rows, H, 128] views of the activations, staged into the workspace
+// when the caller's tensors are fp32 or narrower than 128.
+struct Acts {
+  const __nv_bfloat16 *q, *k, *v, *kt, *vt;
+};
+
+int stage_one(const Plan& P, const void* src, int64_t rows, void* dst, cudaStream_t st) {
+  if (rows == 0) return VDN_OK;
+  const int64_t rh = rows * P.H;
+  const int64_t units = rh * (kDPad / 8);
+  const int threads = 256;
+  const int blocks = (int)imin((int)((units + threads - 1) / threads), 148 * 16);
+  if (P.dtype == VDN_F32)
+    k_pad_to_bf16<float><<<blocks, threads, 0, st>>>(static_cast<const float*>(src),
+                                                     static_cast<__nv_bfloat16*>(dst), rh, P.d);
+  else
+    k_pad_to_bf16<__nv_bfloat16><<<blocks, threads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), rh, P.d);
+  return VDN_OK;
+}
+
+Acts stage_inputs(const Plan& P, const void* q, const void* k, const void* v, const void* kt,
+                  const void* vt, uint8_t* ws, cudaStream_t st, bool need_q, bool need_kv) {
+  Acts a;
+  if (!P.staged) {
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.kt = static_cast<const __nv_bfloat16*>(kt);
+    a.vt = static_cast<const __nv_bfloat16*>(vt);
+    return a;
+  }
+  a.q = reinterpret_cast<const __nv_bfloat16*>(ws + P.o_q);
+  a.k = reinterpret_cast<const __nv_bfloat16*>(ws + P.o_k);
+  a.v = reinterpret_cast<const __nv_bfloat16*>(ws + P.o_v);
+  a.kt = reinterpret_cast<const __nv_bfloat16*>(ws + P.o_kt);
+  a.vt = reinterpret_cast<const __nv_bfloat16*>(ws + P.o_vt);
+  if (need_q) stage_one(P, q, P.N, ws + P.o_q, st);
+  if (need_kv) {
+    stage_one(P, k, P.N, ws + P.o_k, st);
+    stage_one(P, v, P.N, ws + P.o_v, st);
+    stage_one(P, kt, P.T, ws + P.o_kt, st);
+    stage_one(P, vt, P.T, ws + P.o_vt, st);
+  }
+  return a;
+}
+
+// TMA maps; empty tensors get a never-dereferenced map over the workspace.
+bool act_map(CUtensorMap* m, const void* ptr, int64_t rows, const Plan& P, int box, void* dummy) {
+  if (rows == 0) return map_act(m, dummy, 1, P.H, box);
+  return map_act(m, ptr, rows, P.H, box);
+}
+
+int launch_vda(const Plan& P, const Acts& a, uint8_t* ws, cudaStream_t st, float* text_out,
+               float* fwd_out, float* bwd_out) {
+  CUtensorMap tk, tv, tkt, tvt, tw;
+  if (!act_map(&tk, a.k, P.N, P, 64, ws + P.o_C) || !act_map(&tv, a.v, P.N, P, 64, ws + P.o_C) ||
+      !act_map(&tkt, a.kt, P.T, P, 64, ws + P.o_C) ||
+      !act_map(&tvt, a.vt, P.T, P, 64, ws + P.o_C) ||
+      !map_mat(&tw, ws + P.o_W, (int64_t)(P.F - 1) * P.H * 128))
+    return VDN_ERR_CUDA;
+  GramParams gp;
+  gp.off = P.off_dev;
+  gp.F = P.F;
+  gp.T = P.T;
+  gp.H = P.H;
+  gp.lambda = P.lambda;
+  gp.Cmat = reinterpret_cast<float*>(ws + P.o_C);
+  gp.Wmat = reinterpret_cast<float*>(ws + P.o_W);
+  k_vda_gram_inv<<<dim3(P.F - 1, P.H), kGramThreads, kGramSmemBytes, st>>>(tk, tv, tkt, tvt, gp);
+  ScanParams sp;
+  sp.Cmat = gp.Cmat;
+  sp.F = P.F;
+  sp.H = P.H;
+  sp.bf = P.bf;
+  sp.nb = P.nb;
+  sp.lambda = P.lambda;
+  sp.Rpart = reinterpret_cast<float*>(ws + P.o_R);
+  sp.text_out = text_out;
+  sp.fwd_out = fwd_out;
+  sp.bwd_out = bwd_out;
+  sp.d_out = P.d;
+  k_vda_scan<<<dim3(2, P.H), kScanThreads, kScanSmemBytes, st>>>(tw, sp);
+  return VDN_OK;
+}
+
+int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int64_t o_row,
+               int d_store, float* lse, cudaStream_t st) {
+  if (P.N == 0) return VDN_OK;
+  CUtensorMap tq, tk, tv, tkt, tvt;
+  if (!act_map(&tq, a.q, P.N, P, 128, ws + P.o_C) || !act_map(&tk, a.k, P.N, P, 128, ws + P.o_C) ||
+      !act_map(&tv, a.v, P.N, P, 128, ws + P.o_C) ||
+      !act_map(&tkt, a.kt, P.T, P, 128, ws + P.o_C) ||
+      !act_map(&tvt, a.vt, P.T, P, 128, ws + P.o_C))
+    return VDN_ERR_CUDA;
+  BsaParams bp;
+  bp.off = P.off_dev;
+  bp.F = P.F;
+  bp.T = P.T;
+  bp.H = P.H;
+  bp.bf = P.bf;
+  bp.N = P.N;
+  bp.scale_log2 = 1.4426950408889634f / sqrtf((float)P.d);
+  bp.o = o;
+  bp.o_row_stride = o_row;
+  bp.d_store = d_store;
+  bp.lse = lse;
+  k_bsa_fwd<<<dim3(P.max_qtiles, P.nb, P.H), kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt,
+                                                                              tvt, bp);
+  return VDN_OK;
+}
+
+int launch_merge(const Plan& P, const __nv_bfloat16* qb, const float* RA, const float* RB, int r_d,
+                 const __nv_bfloat16* o_soft, int64_t os_row, int os_head, const void* g_s,
+                 const void* g_l, const float* rms_w, void* out, uint8_t* ws, cudaStream_t st) {
+  if (P.N == 0) return VDN_OK;
+  CUtensorMap tq;
+  if (!act_map(&tq, qb, P.N, P, 128, ws + P.o_C)) return VDN_ERR_CUDA;
+  MergeParams mp;
+  mp.off = P.off_dev;
+  mp.F = P.F;
+  mp.H = P.H;
+  mp.bf = P.bf;
+  mp.N = P.N;
+  mp.d = P.d;
+  mp.RA = RA;
+  mp.RB = RB;
+  mp.r_d = r_d;
+  mp.o_soft = o_soft;
+  mp.os_row = os_row;
+  mp.os_head = os_head;
+  mp.g_s = g_s;
+  mp.g_l = g_l;
+  mp.gate_f32 = (P.dtype == VDN_F32);
+  mp.rms_w = rms_w;
+  mp.eps = P.eps;
+  mp.out = out;
+  mp.out_f32 = (P.dtype == VDN_F32);
+  const int gx = (P.max_qtiles + kMergeTiles - 1) / kMergeTiles;
+  k_readout_merge<<<dim3(gx, P.nb, P.H), kMergeThreads, kMergeSmemBytes, st>>>(tq, mp);
+  return VDN_OK;
+}
+
+int finish(int rc) {
+  if (rc != VDN_OK) return rc;
+  return cudaGetLastError() == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
+int common_checks(const Plan& P, void* ws, size_t ws_bytes) {
+  if (ws == nullptr || ws_bytes < P.total) return VDN_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(ws)) return VDN_ERR_MISALIGNED;
+  if (!set_smem_attrs()) return VDN_ERR_CUDA;
+  if (!encode_fn()) return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
+int check_ptrs(std::initializer_list<const void*> must, std::initializer_list<const void*> text,
+               int T) {
+  for (const void* p : must) {
+    if (p == nullptr) return VDN_ERR_INVALID_ARG;
+    if (!aligned16(p)) return VDN_ERR_MISALIGNED;
+  }
+  if (T > 0) {
+    for (const void* p : text) {
+      if (p == nullptr) return VDN_ERR_INVALID_ARG;
+      if (!aligned16(p)) return VDN_ERR_MISALIGNED;
+    }
+  }
+  return VDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t vdn_workspace_bytes(const vdn_shape_t* shape) {
+  Plan P;
+  if (make_plan(shape, &P) != VDN_OK) return 0;
+  return P.total;
+}
+
+int vdn_hybrid_attn_fwd(const vdn_shape_t* shape, const void* q, const void* k, const void* v,
+                        const void* kt, const void* vt, const void* g_s, const void* g_l,
+                        const float* rms_w, void* out, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (P.N == 0) return VDN_OK;  // no query tokens: nothing to write
+  rc = check_ptrs({q, k, v, g_s, g_l, rms_w, out}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, true, true);
+  rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr);
+  if (rc == VDN_OK)
+    rc = launch_bsa(P, a, ws, reinterpret_cast<__nv_bfloat16*>(ws + P.o_osoft),
+                    (int64_t)P.H * kDPad, kDPad, nullptr, st);
+  const float* R = reinterpret_cast<const float*>(ws + P.o_R);
+  if (rc == VDN_OK)
+    rc = launch_merge(P, a.q, R, R + (size_t)P.nb * P.H * 128 * 128, 128,
+                      reinterpret_cast<const __nv_bfloat16*>(ws + P.o_osoft), (int64_t)P.H * kDPad,
+                      kDPad, g_s, g_l, rms_w, out, ws, st);
+  return finish(rc);
+}
+
+int vdn_vda_scan(const vdn_shape_t* shape, const void* k, const void* v, const void* kt,
+                 const void* vt, float* read_states, float* text_state, float* fwd_states,
+                 float* bwd_states, void* workspace, size_t ws_bytes, void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (P.N > 0) rc = check_ptrs({k, v, read_states}, {kt, vt}, P.T);
+  else rc = check_ptrs({read_states}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  for (const void* p : {(const void*)text_state, (const void*)fwd_states, (const void*)bwd_states})
+    if (p != nullptr && !aligned16(p)) return VDN_ERR_MISALIGNED;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const Acts a = stage_inputs(P, nullptr, k, v, kt, vt, ws, st, false, true);
+  rc = launch_vda(P, a, ws, st, text_state, fwd_states, bwd_states);
+  if (rc != VDN_OK) return finish(rc);
+  // read_states [nb][H][d][d] = fwd part + bwd part (leading d x d block)
+  const float* R = reinterpret_cast<const float*>(ws + P.o_R);
+  const size_t part = (size_t)P.nb * P.H * 128 * 128;
+  const int d = P.d;
+  const int64_t n = (int64_t)P.nb * P.H * d * d;
+  k_sum_states<<<(int)((n + 255) / 256), 256, 0, st>>>(R, R + part, read_states, n, d);
+  return finish(VDN_OK);
+}
+
+int vdn_gate_merge(const vdn_shape_t* shape, const void* q, const float* read_states,
+                   const void* o_soft, const void* g_s, const void* g_l, const float* rms_w,
+                   void* out, void* workspace, size_t ws_bytes, void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (P.N == 0) return VDN_OK;
+  rc = check_ptrs({q, read_states, o_soft, g_s, g_l, rms_w, out}, {}, 0);
+  if (rc != VDN_OK) return rc;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const Acts a = stage_inputs(P, q, nullptr, nullptr, nullptr, nullptr, ws, st, true, false);
+  rc = launch_merge(P, a.q, read_states, nullptr, P.d, static_cast<const __nv_bfloat16*>(o_soft),
+                    (int64_t)P.H * P.d, P.d, g_s, g_l, rms_w, out, ws, st);
+  return finish(rc);
+}
+
+int vdn_bsa_fwd(const vdn_shape_t* shape, const void* q, const void* k, const void* v,
+                const void* kt, const void* vt, void* o_soft, float* lse, void* workspace,
+                size_t ws_bytes, void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (P.N == 0) return VDN_OK;
+  rc = check_ptrs({q, k, v, o_soft}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  if (lse != nullptr && !aligned16(lse)) return VDN_ERR_MISALIGNED;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, true, true);
+  rc = launch_bsa(P, a, ws, static_cast<__nv_bfloat16*>(o_soft), (int64_t)P.H * P.d, P.d, lse, st);
+  return finish(rc);
+}
+
+int vdn_pair_audit(const vdn_shape_t* shape, int64_t* soft_pairs, int64_t* lin_pairs,
+                   void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (soft_pairs == nullptr || lin_pairs == nullptr) return VDN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(soft_pairs, 0, sizeof(int64_t) * P.F * (P.F + 1), st) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  if (P.max_qtiles > 0)
+    k_pair_audit_soft<<<dim3(P.max_qtiles, P.nb), 128, 0, st>>>(
+        P.off_dev, P.F, P.T, P.bf, reinterpret_cast<unsigned long long*>(soft_pairs));
+  k_pair_audit_lin<<<P.F, 128, 0, st>>>(P.off_dev, P.F, P.bf,
+                                         reinterpret_cast<unsigned long long*>(lin_pairs));
+  return finish(VDN_OK);
+}
+
+int vdn_get_device_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return VDN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, vdn::g_device_error, sizeof(int)) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(vdn::g_device_error, &zero, sizeof(int)) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  if (v == kDevErrWaitTimeout) return VDN_ERR_DEVICE_TIMEOUT;
+  return v == 0 ? VDN_OK : VDN_ERR_DEVICE;
+}
+
+const char* vdn_error_string(int code) {
+  switch (code) {
+    case VDN_OK: return "ok";
+    case VDN_ERR_INVALID_ARG: return "invalid argument";
+    case VDN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case VDN_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case VDN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case VDN_ERR_CUDA: return "CUDA launch or driver error";
+    case VDN_ERR_DEVICE_TIMEOUT: return "device-side bounded wait expired";
+    case VDN_ERR_DEVICE: return "device-side error";
+    default: return "unknown error";
+  }
+}
+
+}  // extern "C"
