@@ -141,6 +141,23 @@ int vdn_bsa_fwd(const vdn_shape_t* shape, const void* q, const void* k,
 int vdn_pair_audit(const vdn_shape_t* shape, int64_t* soft_pairs,
                    int64_t* lin_pairs, void* stream);
 
+/* Same results as vdn_vda_scan, for callers that cannot provide a workspace
+ * (no paper counterpart: this is a deployment variant). Its scratch is a
+ * 64 MiB array inside the library, resident on every GPU that loads the
+ * library until the process exits; the call itself allocates nothing.
+ * Limit: 128 KiB x H x (F - 1) for the per-frame matrices, plus
+ * 128 KiB x H x ceil(F / block_frames) for the read states, plus (fp32 or
+ * d < 128 inputs only) 256 B x H x (2N + 2T) of staged keys/values must fit
+ * in 64 MiB; larger shapes return VDN_ERR_WORKSPACE_TOO_SMALL. The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress), so
+ * make that first call before any stream capture. All calls share the one
+ * array: calls that overlap on the GPU (other streams, other host threads)
+ * race and must be ordered by the caller. */
+int vdn_vda_scan_noalloc(const vdn_shape_t* shape, const void* k, const void* v,
+                         const void* kt, const void* vt, float* read_states,
+                         float* text_state, float* fwd_states, float* bwd_states,
+                         void* stream);
+
 /* Synchronises the current device, returns VDN_OK or the first device-side
  * error recorded since the last call (VDN_ERR_DEVICE_TIMEOUT for an expired
  * bounded wait), and clears it. */

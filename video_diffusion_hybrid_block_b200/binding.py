@@ -59,6 +59,7 @@ _SIGS = {
     "vdn_gate_merge": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
     "vdn_bsa_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
     "vdn_pair_audit": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t), _P, _P, _P]),
+    "vdn_vda_scan_noalloc": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 8 + [_P]),
     "vdn_get_device_error": (ctypes.c_int, []),
     "vdn_error_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -164,6 +165,17 @@ def vdn_vda_scan(shape: Shape, k, v, kt, vt, read_states, text_state, fwd_states
         _ptr(fwd_states), _ptr(bwd_states), _ptr(workspace),
         _nbytes(workspace, ws_bytes), _stream(stream))
     _check(rc, "vdn_vda_scan")
+    return read_states
+
+
+def vdn_vda_scan_noalloc(shape: Shape, k, v, kt, vt, read_states, text_state, fwd_states,
+                         bwd_states, stream=None):
+    """vdn_vda_scan without a workspace argument: the library's built-in
+    64 MiB device scratch is used instead (see include/vdn.h for the limit)."""
+    rc = load_library().vdn_vda_scan_noalloc(
+        shape.ref, _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(read_states), _ptr(text_state),
+        _ptr(fwd_states), _ptr(bwd_states), _stream(stream))
+    _check(rc, "vdn_vda_scan_noalloc")
     return read_states
 
 

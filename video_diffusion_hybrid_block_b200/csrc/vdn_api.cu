@@ -477,3 +477,86 @@ const char* vdn_error_string(int code) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Linear-branch states without a caller-provided workspace.
+//
+// Some callers cannot hand this library a workspace: code that runs where
+// cudaMalloc is not allowed or not wanted (a host function enqueued with
+// cudaLaunchHostFunc may not call CUDA APIs that allocate; a serving loop
+// whose latency budget cannot absorb the implicit synchronisation of
+// cudaMalloc; a plug-in living inside a process whose memory is owned by
+// another allocator it has no handle to). For them, vdn_vda_scan_noalloc
+// keeps its scratch (per-frame C and W matrices, read-state halves and, for
+// fp32 or d < 128 inputs, the staged bf16 keys/values) in one file-scope
+// device array of kNoAllocScratchBytes. Every GPU that loads this library
+// holds that array until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)64 << 20;  // 64 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device. In host code
+// the symbol itself is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch_address(uint8_t** out) {
+  static uint8_t* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return VDN_ERR_CUDA;
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return VDN_ERR_CUDA;
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = addr[dev];
+  return VDN_OK;
+}
+
+}  // namespace
+
+extern "C" int vdn_vda_scan_noalloc(const vdn_shape_t* shape, const void* k, const void* v,
+                                    const void* kt, const void* vt, float* read_states,
+                                    float* text_state, float* fwd_states, float* bwd_states,
+                                    void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (P.N > 0) rc = check_ptrs({k, v, read_states}, {kt, vt}, P.T);
+  else rc = check_ptrs({read_states}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  for (const void* p : {(const void*)text_state, (const void*)fwd_states, (const void*)bwd_states})
+    if (p != nullptr && !aligned16(p)) return VDN_ERR_MISALIGNED;
+  // Scratch layout inside the static array: C, W, read-state halves, then
+  // the staged keys/values when the inputs need narrowing or padding.
+  Plan S = P;
+  const size_t mat = align256((size_t)(P.F - 1) * P.H * 128 * 128 * 4);
+  const size_t act = P.staged ? align256((size_t)P.N * P.H * kDPad * 2) : 0;
+  const size_t txt = P.staged ? align256((size_t)P.T * P.H * kDPad * 2) : 0;
+  S.o_C = 0;
+  S.o_W = mat;
+  S.o_R = 2 * mat;
+  S.o_k = S.o_R + align256((size_t)2 * P.nb * P.H * 128 * 128 * 4);
+  S.o_v = S.o_k + act;
+  S.o_kt = S.o_v + act;
+  S.o_vt = S.o_kt + txt;
+  S.o_q = S.o_osoft = 0;  // not used by the scan
+  S.total = S.o_vt + txt;
+  if (S.total > kNoAllocScratchBytes) return VDN_ERR_WORKSPACE_TOO_SMALL;
+  uint8_t* scratch = nullptr;
+  rc = noalloc_scratch_address(&scratch);
+  if (rc != VDN_OK) return rc;
+  if (!set_smem_attrs() || !encode_fn()) return VDN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Nothing in the scratch has to start at zero: every region is written in
+  // full by this call before it is read.
+  const Acts a = stage_inputs(S, nullptr, k, v, kt, vt, scratch, st, false, true);
+  rc = launch_vda(S, a, scratch, st, text_state, fwd_states, bwd_states);
+  if (rc != VDN_OK) return finish(rc);
+  const float* R = reinterpret_cast<const float*>(scratch + S.o_R);
+  const size_t part = (size_t)P.nb * P.H * 128 * 128;
+  const int64_t n = (int64_t)P.nb * P.H * P.d * P.d;
+  k_sum_states<<<(int)((n + 255) / 256), 256, 0, st>>>(R, R + part, read_states, n, P.d);
+  return finish(VDN_OK);
+}
