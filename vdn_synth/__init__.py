@@ -6,8 +6,8 @@ oracle (``oracle/``) and the CUDA path (``video_diffusion_hybrid_block_b200``)
 consume what it returns, and neither imports the other.
 
 Workloads (frame grid, token counts, head counts) are synthetic stand-ins for
-the pages' "a dozen-plus latent frames with over a thousand latent tokens each,
-plus text tokens" at 768p (VDN-MiniMax-H3 on openi.cn, section
+the clips the pages describe (somewhat more than ten latent frames, each with
+more than a thousand latent tokens, plus text tokens) at 768p (VDN-MiniMax-H3 on openi.cn, section
 "技术原理：局部精确、远程压缩"); the pages name no dataset or benchmark suite.
 
 Recipe (numpy PCG64 ``default_rng(seed)``, all draws float32, in this order):
