@@ -6,18 +6,31 @@
 // (openi.cn), 技术原理：局部精确、远程压缩; nav.superapi.store page, Technical
 // Principles, Local Softmax Branch / Text Dual-Branch Injection].
 //
-// One CTA = one 128-row query tile of one block and one head. Key tiles are
-// enumerated from the block's key segments (layer_plan.cuh), so tiles outside
-// the allowed set are never loaded; only the ragged last tile of each segment
-// is masked column-wise. Warp roles:
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); online
-//              softmax in the exp2 domain with a lazily updated running max
-//              (O and l are rescaled only when the max grows by > 2^8);
-//              writes P (bf16) to shared memory; final 1/l and bf16 store.
-//   warp 4     TMA producer: Q once, then K and V tiles (2-stage ring).
-//   warp 5     MMA issuer: S = Q K^T into a double-buffered TMEM S, then
-//              O += P V into TMEM O, committing to mbarriers.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384).
+// One CTA = two 128-row query tiles (256 consecutive rows of one block) of one
+// head. Key tiles are enumerated from the block's key segments
+// (layer_plan.cuh), so tiles outside the allowed set are never loaded; only
+// the ragged last tile of each segment is masked column-wise. Both query
+// tiles share every K/V tile. Warp roles (384 threads, 3 warpgroups):
+//   warps 0-3  softmax of query tile 0 (thread r owns row r = TMEM lane r)
+//   warps 4-7  softmax of query tile 1
+//   warp 8     TMA producer: Q0, Q1 once, then K and V tiles (2-stage rings)
+//   warp 9     MMA issuer (one thread); warps 10-11 idle
+// Registers: launched at 168 per thread (384 x 168 = 64512); the producer
+// warpgroup drops to 72 and the two softmax warpgroups rise to 216
+// (128 x (216 + 216 + 72) = 64512), enough to hold a full 128-column S row.
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// P_i (bf16, packed in pairs) overwrites the first 64 columns of S_i and is
+// consumed from TMEM by the PV contraction (A operand in TMEM), so P never
+// touches shared memory. MMA issue order per key tile j:
+//   PV0(j), QK0(j+1), PV1(j), QK1(j+1)
+// so while softmax i works on S_i(j+1), the tensor core runs the other tile's
+// PV and QK. Contractions issued by one thread execute in issue order, so
+// QK_i(j+1) may overwrite S_i right after PV_i(j) read P_i from it; and the
+// commit that signals S_i(j+1) also covers PV_i(j), so the softmax owns O_i
+// (for a rescale) from then until it hands over P_i(j+1).
+// Online softmax in the exp2 domain with a lazily updated running max: O and
+// the row sum are rescaled only when the tile max exceeds the max in use by
+// more than 8 (a factor 256), which keeps every P <= 256.
 #pragma once
 
 #include "layer_plan.cuh"
@@ -25,75 +38,63 @@
 
 namespace vdn {
 
-constexpr int kBsaThreads = 192;
-constexpr uint32_t kBsaSmemQ = 0;
-constexpr uint32_t kBsaSmemK = 32768;          // 2 stages x 32 KB
-constexpr uint32_t kBsaSmemV = 32768 * 3;      // 2 stages x 32 KB
-constexpr uint32_t kBsaSmemP = 32768 * 5;      // 32 KB
-constexpr uint32_t kBsaSmemBytes = 32768 * 6 + 1024;  // + alignment slack
+constexpr int kBsaThreads = 384;
+constexpr int kBsaRegsSoftmax = 216;
+constexpr int kBsaRegsProducer = 72;
+constexpr uint32_t kBsaSmemQ = 0;               // Q0, Q1: 2 x 32 KB
+constexpr uint32_t kBsaSmemK = 2 * 32768;       // 2 stages x 32 KB
+constexpr uint32_t kBsaSmemV = 4 * 32768;       // 2 stages x 32 KB
+constexpr uint32_t kBsaSmemBytes = 6 * 32768 + 1024;  // + alignment slack
+constexpr int kBsaRowsPerCta = 2 * kTile;
 
 struct BsaParams {
   const int32_t* off;  // [F+1] device
   int F, T, H, bf, N;
-  float scale_log2;    // log2(e) / sqrt(d)
-  __nv_bfloat16* o;    // o_soft output base
+  float scale_log2;      // log2(e) / sqrt(d)
+  __nv_bfloat16* o;      // o_soft output base
   int64_t o_row_stride;  // elements between consecutive tokens
-  int d_store;         // leading columns of each head row to store
-  float* lse;          // optional [H][N]
+  int d_store;           // leading columns of each head row to store
+  float* lse;            // optional [H][N]
 };
 
 __global__ void __launch_bounds__(kBsaThreads, 1)
     k_bsa_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkt,
               const __grid_constant__ CUtensorMap tvt, const BsaParams p) {
-  const int tile = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
+  const int pair = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
   int q0, q1;
   block_rows(p.off, p.F, p.bf, b, q0, q1);
-  const int qs = q0 + tile * kTile;
+  const int qs = q0 + pair * kBsaRowsPerCta;
   if (qs >= q1) return;  // uniform over the CTA, before any resource is taken
-  const int qrows = imin(kTile, q1 - qs);
   const KeySegs segs = key_segments(p.off, p.F, p.bf, p.T, b);
   const int nkt = segs_tiles(segs);
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_q, bar_kf[2], bar_ke[2], bar_vf[2], bar_ve[2], bar_sf[2],
-      bar_sfree[2], bar_p, bar_o;
+  __shared__ uint64_t bar_q, bar_kf[2], bar_ke[2], bar_vf[2], bar_ve[2], bar_sf[2], bar_pf[2],
+      bar_of[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sQ = base + kBsaSmemQ;
-  const uint32_t sK[2] = {base + kBsaSmemK, base + kBsaSmemK + 32768};
-  const uint32_t sV[2] = {base + kBsaSmemV, base + kBsaSmemV + 32768};
-  const uint32_t sP = base + kBsaSmemP;
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t q_full = smem_u32(&bar_q);
-  const uint32_t k_full[2] = {smem_u32(&bar_kf[0]), smem_u32(&bar_kf[1])};
-  const uint32_t k_empty[2] = {smem_u32(&bar_ke[0]), smem_u32(&bar_ke[1])};
-  const uint32_t v_full[2] = {smem_u32(&bar_vf[0]), smem_u32(&bar_vf[1])};
-  const uint32_t v_empty[2] = {smem_u32(&bar_ve[0]), smem_u32(&bar_ve[1])};
-  const uint32_t s_full[2] = {smem_u32(&bar_sf[0]), smem_u32(&bar_sf[1])};
-  const uint32_t s_free[2] = {smem_u32(&bar_sfree[0]), smem_u32(&bar_sfree[1])};
-  const uint32_t p_full = smem_u32(&bar_p);
-  const uint32_t o_done = smem_u32(&bar_o);
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(k_full[i], 1);
-      mbar_init(k_empty[i], 1);
-      mbar_init(v_full[i], 1);
-      mbar_init(v_empty[i], 1);
-      mbar_init(s_full[i], 1);
-      mbar_init(s_free[i], 128);
+      mbar_init(smem_u32(&bar_kf[i]), 1);
+      mbar_init(smem_u32(&bar_ke[i]), 1);
+      mbar_init(smem_u32(&bar_vf[i]), 1);
+      mbar_init(smem_u32(&bar_ve[i]), 1);
+      mbar_init(smem_u32(&bar_sf[i]), 1);
+      mbar_init(smem_u32(&bar_pf[i]), 128);
+      mbar_init(smem_u32(&bar_of[i]), 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&tmem_slot), 512);
     tmem_relinquish();
   }
@@ -102,16 +103,21 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
-
-  if (warp == 4) {
+  // Each role's code sits inside the branch that set its register budget, so
+  // no path joins two budgets before the common teardown.
+  if (warp >= 8) {
+  regs_dealloc<kBsaRegsProducer>();
+  if (warp == 8) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      mbar_arrive_expect_tx(q_full, 32768);
+      mbar_arrive_expect_tx(q_full, 2 * 32768);
       tma_load_3d(sQ, &tq, q_full, 0, h, qs);
       tma_load_3d(sQ + 16384, &tq, q_full, 64, h, qs);
+      tma_load_3d(sQ + 32768, &tq, q_full, 0, h, qs + kTile);
+      tma_load_3d(sQ + 49152, &tq, q_full, 64, h, qs + kTile);
       for (int j = 0; j < nkt; ++j) {
         if (*abort_v) break;
         const int st = j & 1;
@@ -120,167 +126,205 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         segs_tile(segs, j, src, row0, valid);
         const CUtensorMap* mk = src ? &tkt : &tk;
         const CUtensorMap* mv = src ? &tvt : &tv;
-        if (!mbar_wait(k_empty[st], ph ^ 1)) { *abort_v = 1; break; }
-        mbar_arrive_expect_tx(k_full[st], 32768);
-        tma_load_3d(sK[st], mk, k_full[st], 0, h, row0);
-        tma_load_3d(sK[st] + 16384, mk, k_full[st], 64, h, row0);
-        if (!mbar_wait(v_empty[st], ph ^ 1)) { *abort_v = 1; break; }
-        mbar_arrive_expect_tx(v_full[st], 32768);
-        tma_load_3d(sV[st], mv, v_full[st], 0, h, row0);
-        tma_load_3d(sV[st] + 16384, mv, v_full[st], 64, h, row0);
+        const uint32_t sK = base + kBsaSmemK + (uint32_t)st * 32768u;
+        const uint32_t sV = base + kBsaSmemV + (uint32_t)st * 32768u;
+        const uint32_t kf = smem_u32(&bar_kf[st]), vf = smem_u32(&bar_vf[st]);
+        if (!mbar_wait(smem_u32(&bar_ke[st]), ph ^ 1)) { *abort_v = 1; break; }
+        mbar_arrive_expect_tx(kf, 32768);
+        tma_load_3d(sK, mk, kf, 0, h, row0);
+        tma_load_3d(sK + 16384, mk, kf, 64, h, row0);
+        if (!mbar_wait(smem_u32(&bar_ve[st]), ph ^ 1)) { *abort_v = 1; break; }
+        mbar_arrive_expect_tx(vf, 32768);
+        tma_load_3d(sV, mv, vf, 0, h, row0);
+        tma_load_3d(sV + 16384, mv, vf, 64, h, row0);
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // -------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, 128, false, false);
       const uint32_t idO = idesc_bf16(128, 128, false, true);
-      bool ok = mbar_wait(q_full, 0);
-      tc_fence_after();
-      // S(j) = Q K(j)^T into TMEM buffer j&1
-      auto issue_qk = [&](int j) -> bool {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(k_full[st], ph)) return false;
-        if (!mbar_wait(s_free[st], ph ^ 1)) return false;
-        tc_fence_after();
-        const uint32_t dS = tmem + (uint32_t)(st * 128);
+      // S_i = Q_i K^T for key tile in K stage st
+      auto qk = [&](int i, int st) {
+        const uint32_t sQi = sQ + (uint32_t)i * 32768u;
+        const uint32_t sK = base + kBsaSmemK + (uint32_t)st * 32768u;
+        const uint32_t dS = tmem + (uint32_t)(i * 128);
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           const uint32_t ko = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
-          umma_bf16_ss(dS, sdesc_sw128(sQ + ko, 16, 1024), sdesc_sw128(sK[st] + ko, 16, 1024),
-                       idS, s > 0 ? 1u : 0u);
+          umma_bf16_ss(dS, sdesc_sw128(sQi + ko, 16, 1024), sdesc_sw128(sK + ko, 16, 1024), idS,
+                       s > 0 ? 1u : 0u);
         }
-        umma_commit(k_empty[st]);
-        umma_commit(s_full[st]);
-        return true;
+        umma_commit(smem_u32(&bar_sf[i]));
       };
-      if (ok) ok = issue_qk(0);
+      // O_i += P_i V with P_i read from the first 64 TMEM columns of S_i
+      auto pv = [&](int i, int st, bool acc) {
+        const uint32_t sV = base + kBsaSmemV + (uint32_t)st * 32768u;
+        const uint32_t aP = tmem + (uint32_t)(i * 128);
+        const uint32_t dO = tmem + 256u + (uint32_t)(i * 128);
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          umma_bf16_ts(dO, aP + (uint32_t)(s * 8), sdesc_sw128(sV + (uint32_t)(s * 2048), 16384, 1024),
+                       idO, (acc || s > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(q_full, 0) && mbar_wait(smem_u32(&bar_kf[0]), 0);
+      if (ok) {
+        tc_fence_after();
+        qk(0, 0);
+        qk(1, 0);
+        umma_commit(smem_u32(&bar_ke[0]));
+      }
       for (int j = 0; ok && j < nkt; ++j) {
         if (*abort_v) { ok = false; break; }
-        if (j + 1 < nkt && !issue_qk(j + 1)) { ok = false; break; }
         const int st = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(p_full, (uint32_t)(j & 1))) { ok = false; break; }
-        if (!mbar_wait(v_full[st], ph)) { ok = false; break; }
+        const int st1 = (j + 1) & 1;
+        const uint32_t ph1 = ((j + 1) >> 1) & 1;
+        const bool more = j + 1 < nkt;
+        if (!mbar_wait(smem_u32(&bar_vf[st]), ph)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&bar_pf[0]), (uint32_t)(j & 1))) { ok = false; break; }
         tc_fence_after();
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          umma_bf16_ss(tmem + 256, sdesc_sw128(sP + (uint32_t)((s >> 2) * 16384 + (s & 3) * 32), 16, 1024),
-                       sdesc_sw128(sV[st] + (uint32_t)(s * 2048), 16384, 1024), idO,
-                       (j > 0 || s > 0) ? 1u : 0u);
+        pv(0, st, j > 0);
+        if (!more) umma_commit(smem_u32(&bar_of[0]));
+        if (more) {
+          if (!mbar_wait(smem_u32(&bar_kf[st1]), ph1)) { ok = false; break; }
+          tc_fence_after();
+          qk(0, st1);
         }
-        umma_commit(v_empty[st]);
-        umma_commit(o_done);
+        if (!mbar_wait(smem_u32(&bar_pf[1]), (uint32_t)(j & 1))) { ok = false; break; }
+        tc_fence_after();
+        pv(1, st, j > 0);
+        umma_commit(smem_u32(&bar_ve[st]));
+        if (!more) umma_commit(smem_u32(&bar_of[1]));
+        if (more) {
+          qk(1, st1);
+          umma_commit(smem_u32(&bar_ke[st1]));
+        }
       }
       if (!ok) *abort_v = 1;
     }
     __syncwarp();
+  }
   } else {
+    regs_alloc<kBsaRegsSoftmax>();
     // ---------------------------------------------------- softmax warps --
-    const int r = threadIdx.x;  // query row within the tile == TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    float m_use = 0.f, l_sum = 0.f;
+    const int tile = warp >> 2;             // query tile of this warpgroup
+    const int r = threadIdx.x & 127;        // row within the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (uint32_t)(tile * 128);
+    const uint32_t tO = tmem + lane_base + 256u + (uint32_t)(tile * 128);
+    const uint32_t s_full = smem_u32(&bar_sf[tile]);
+    const uint32_t p_full = smem_u32(&bar_pf[tile]);
+    const float scale = p.scale_log2;
+    float m_use = 0.f;
+    float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
     bool ok = true;
     for (int j = 0; j < nkt; ++j) {
       if (*abort_v) { ok = false; break; }
-      const int st = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
       int src, row0, valid;
       segs_tile(segs, j, src, row0, valid);
-      if (!mbar_wait(s_full[st], ph)) { ok = false; break; }
+      if (!mbar_wait(s_full, (uint32_t)(j & 1))) { ok = false; break; }
       tc_fence_after();
       uint32_t s[128];
-      tmem_ld128(tmem + lane_base + (uint32_t)(st * 128), s);
+      tmem_ld128(tS, s);
       tmem_ld_wait128(s);
-      tc_fence_before();
-      mbar_arrive(s_free[st]);
-
-      float mloc = -INFINITY;
+      if (valid < 128) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        float x = __uint_as_float(s[i]) * p.scale_log2;
-        x = (i < valid) ? x : -INFINITY;
-        s[i] = __float_as_uint(x);
-        mloc = fmaxf(mloc, x);
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) s[c] = __float_as_uint(-INFINITY);
       }
-      bool need = false;
-      float factor = 1.f;
+      // tile row max of the raw scores (scale > 0 keeps the order)
+      float mx = fmax3(__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]));
+#pragma unroll
+      for (int c = 3; c < 127; c += 2)
+        mx = fmax3(mx, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+      mx = fmaxf(mx, __uint_as_float(s[127]));
+      const float m_tile = mx * scale;
       if (j == 0) {
-        m_use = mloc;
-      } else if (mloc > m_use + 8.f) {
-        need = true;
-        factor = ex2_approx(m_use - mloc);
-        m_use = mloc;
-        l_sum *= factor;
-      }
-      float rs = 0.f;
-      uint32_t pk[64];
+        m_use = m_tile;
+      } else {
+        const bool need = m_tile > m_use + 8.f;
+        if (__any_sync(0xffffffffu, need)) {
+          // O_i is idle here: PV_i(j-1) completed before S_i(j) was signalled.
+          const float factor = need ? ex2_approx(m_use - m_tile) : 1.f;
+          if (need) {
+            m_use = m_tile;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float e0 = ex2_approx(__uint_as_float(s[2 * i]) - m_use);
-        const float e1 = ex2_approx(__uint_as_float(s[2 * i + 1]) - m_use);
-        rs += e0 + e1;
-        pk[i] = pack_bf16x2(e0, e1);
-      }
-      l_sum += rs;
-      // PV(j-1) must be done: P buffer is reused and O may be rescaled.
-      if (j > 0 && !mbar_wait(o_done, (uint32_t)((j - 1) & 1))) { ok = false; break; }
-      tc_fence_after();
-      if (__any_sync(0xffffffffu, need)) {
+            for (int a = 0; a < 4; ++a) {
+              lacc[a].x *= factor;
+              lacc[a].y *= factor;
+            }
+          }
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + 256u + (uint32_t)(c * 32), o);
-          tmem_ld_wait(o);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + (uint32_t)(c * 32), o);
+            tmem_ld_wait(o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-          tmem_st32(tmem + lane_base + 256u + (uint32_t)(c * 32), o);
-        }
-        tmem_st_wait();
-      }
-      // P row r -> shared memory, 128B-swizzled K-major (two 64-key chunks)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int i = c * 32 + u * 4;
-          st_shared_v4(sP + (uint32_t)(c * 16384) + sw128_off((uint32_t)r, (uint32_t)u), pk[i],
-                       pk[i + 1], pk[i + 2], pk[i + 3]);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(tO + (uint32_t)(c * 32), o);
+          }
         }
       }
-      fence_proxy_async_smem();
+      // P = exp2(s * scale - m_use), packed to bf16 pairs, written into S_i's
+      // first 64 TMEM columns
+      const float2 sc2 = make_float2(scale, scale);
+      const float2 nm2 = make_float2(-m_use, -m_use);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = half * 64 + 2 * e;
+          const float2 x = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2);
+          const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          lacc[e & 3] = fadd2(lacc[e & 3], pe);
+          pk[e] = pack_bf16x2(pe.x, pe.y);
+        }
+        tmem_st32(tS + (uint32_t)(half * 32), pk);
+      }
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    if (ok && !mbar_wait(o_done, (uint32_t)((nkt - 1) & 1))) ok = false;
+    const float l_sum = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y) +
+                        (lacc[2].x + lacc[2].y) + (lacc[3].x + lacc[3].y);
+    if (ok && !mbar_wait(smem_u32(&bar_of[tile]), 0)) ok = false;
     if (!ok) *abort_v = 1;
     tc_fence_after();
-    uint32_t o[128];
-    tmem_ld128(tmem + lane_base + 256u, o);
-    tmem_ld_wait128(o);
-    if (ok && r < qrows) {
-      const float inv = 1.f / l_sum;
-      __nv_bfloat16* dst = p.o + (int64_t)(qs + r) * p.o_row_stride + (int64_t)h * p.d_store;
+    const int row = qs + tile * kTile + r;
+    const bool store = ok && row < q1;
+    const float inv = 1.f / l_sum;
+    __nv_bfloat16* dst = p.o + (int64_t)row * p.o_row_stride + (int64_t)h * p.d_store;
+    // the TMEM loads are warp-collective: every thread runs them, only the
+    // stores depend on the row
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        if (u * 8 < p.d_store) {
-          uint4 val;
-          val.x = pack_bf16x2(__uint_as_float(o[u * 8 + 0]) * inv, __uint_as_float(o[u * 8 + 1]) * inv);
-          val.y = pack_bf16x2(__uint_as_float(o[u * 8 + 2]) * inv, __uint_as_float(o[u * 8 + 3]) * inv);
-          val.z = pack_bf16x2(__uint_as_float(o[u * 8 + 4]) * inv, __uint_as_float(o[u * 8 + 5]) * inv);
-          val.w = pack_bf16x2(__uint_as_float(o[u * 8 + 6]) * inv, __uint_as_float(o[u * 8 + 7]) * inv);
-          *reinterpret_cast<uint4*>(dst + u * 8) = val;
+    for (int c = 0; c < 4; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + (uint32_t)(c * 32), o);
+      tmem_ld_wait(o);
+      if (store) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (c * 32 + u * 8 < p.d_store) {
+            uint4 val;
+            val.x = pack_bf16x2(__uint_as_float(o[u * 8 + 0]) * inv, __uint_as_float(o[u * 8 + 1]) * inv);
+            val.y = pack_bf16x2(__uint_as_float(o[u * 8 + 2]) * inv, __uint_as_float(o[u * 8 + 3]) * inv);
+            val.z = pack_bf16x2(__uint_as_float(o[u * 8 + 4]) * inv, __uint_as_float(o[u * 8 + 5]) * inv);
+            val.w = pack_bf16x2(__uint_as_float(o[u * 8 + 6]) * inv, __uint_as_float(o[u * 8 + 7]) * inv);
+            *reinterpret_cast<uint4*>(dst + c * 32 + u * 8) = val;
+          }
         }
       }
-      if (p.lse != nullptr)
-        p.lse[(int64_t)h * p.N + qs + r] = (m_use + __log2f(l_sum)) * 0.69314718055994531f;
     }
+    if (store && p.lse != nullptr)
+      p.lse[(int64_t)h * p.N + row] = (m_use + __log2f(l_sum)) * 0.69314718055994531f;
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

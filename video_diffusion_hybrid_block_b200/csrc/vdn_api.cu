@@ -267,8 +267,8 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
   bp.o_row_stride = o_row;
   bp.d_store = d_store;
   bp.lse = lse;
-  k_bsa_fwd<<<dim3(P.max_qtiles, P.nb, P.H), kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt,
-                                                                              tvt, bp);
+  k_bsa_fwd<<<dim3((P.max_qtiles + 1) / 2, P.nb, P.H), kBsaThreads, kBsaSmemBytes, st>>>(
+      tq, tk, tv, tkt, tvt, bp);
   return VDN_OK;
 }
 
