@@ -312,6 +312,53 @@ def cpu_baseline(inp: dict, fl: dict, heads: int) -> dict:
                       f"(all {inp['N']} query rows), pages-scale workload"}
 
 
+def run_profile(args) -> None:
+    """Runs `--steps` launches of one entry point (after `--warmup`) on a
+    workload with optionally fewer heads, for bounded ncu captures."""
+    import torch
+
+    import video_diffusion_hybrid_block_b200 as V
+    import vdn_synth as S
+
+    cfg = dict(S.CONFIGS[args.workload])
+    if args.heads:
+        cfg["H"] = args.heads
+    inp = S.make_inputs_from(cfg["F"], S.frame_sizes(cfg), cfg["T"], cfg["H"], cfg["d"],
+                             dtype=cfg["dtype"], seed=0, k_lowrank=cfg.get("k_lowrank"),
+                             zero_v_every=cfg.get("zero_v_every"))
+    dt = torch.bfloat16 if cfg["dtype"] == "bf16" else torch.float32
+    dev = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to("cuda", dt)
+           for k in ("q", "k", "v", "kt", "vt", "g_s", "g_l")}
+    rms_w = torch.from_numpy(inp["rms_w"]).cuda()
+    shape = V.Shape(inp["off"], inp["T"], inp["H"], inp["d"], inp["block_frames"], inp["lam"],
+                    inp["eps"], V.VDN_BF16 if cfg["dtype"] == "bf16" else V.VDN_F32)
+    ws = V.alloc_workspace(shape)
+    out = torch.empty_like(dev["q"])
+    nb = -(-inp["F"] // inp["block_frames"])
+    R = torch.empty((nb, inp["H"], inp["d"], inp["d"]), device="cuda")
+    o_soft = torch.empty(dev["q"].shape, dtype=torch.bfloat16, device="cuda")
+
+    def once():
+        if args.profile == "layer":
+            V.vdn_hybrid_attn_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"],
+                                  dev["g_s"], dev["g_l"], rms_w, out, ws)
+        elif args.profile == "bsa":
+            V.vdn_bsa_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"], o_soft, None,
+                          ws)
+        else:
+            V.vdn_vda_scan(shape, dev["k"], dev["v"], dev["kt"], dev["vt"], R, None, None, None,
+                           ws)
+
+    for _ in range(args.warmup + args.steps):
+        once()
+    torch.cuda.synchronize()
+    rc = V.vdn_get_device_error()
+    print(json.dumps({"profile": args.profile, "workload": args.workload, "H": inp["H"],
+                      "launches": args.warmup + args.steps, "device_error": rc}))
+    if rc != 0:
+        sys.exit(1)
+
+
 def run_reference(args) -> None:
     world, rank, _ = dist_env()
     if rank != 0:
@@ -361,7 +408,14 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--cpu-heads", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["layer", "bsa", "vda"],
+                    help="only run launches of one entry point (for ncu captures)")
+    ap.add_argument("--workload", default=WORKLOAD, help="workload for --profile")
+    ap.add_argument("--heads", type=int, default=0, help="override head count for --profile")
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args)
+        return
     if args.warmup < 3 and args.impl == "cuda":
         args.warmup = 3
     if args.impl == "reference":

@@ -31,6 +31,15 @@
 // Online softmax in the exp2 domain with a lazily updated running max: O and
 // the row sum are rescaled only when the tile max exceeds the max in use by
 // more than 8 (a factor 256), which keeps every P <= 256.
+//
+// kMerge = true fuses the linear-branch readout and the gated merge into the
+// epilogue: after the last PV_i the MMA thread issues o_lin_i = Q_i R_b into
+// the (now free) S_i columns, with R_b a packed bf16 tile loaded once per CTA;
+// each softmax thread then forms
+//   out = sigmoid(g_s) O/l + sigmoid(g_l) w * o_lin / sqrt(mean(o_lin^2) + eps)
+// for its row ["VDN-MiniMax-H3" (openi.cn), 技术原理, last paragraph;
+// nav.superapi.store page, Gated Fusion Mechanism], so o_soft never goes to
+// HBM and q is not read a second time.
 #pragma once
 
 #include "layer_plan.cuh"
@@ -41,10 +50,15 @@ namespace vdn {
 constexpr int kBsaThreads = 384;
 constexpr int kBsaRegsSoftmax = 216;
 constexpr int kBsaRegsProducer = 72;
+constexpr int kBsaMergeRegsSoftmax = 208;
+constexpr int kBsaMergeRegsProducer = 88;  // 128 x (208 + 208 + 88) = 64512
 constexpr uint32_t kBsaSmemQ = 0;               // Q0, Q1: 2 x 32 KB
 constexpr uint32_t kBsaSmemK = 2 * 32768;       // 2 stages x 32 KB
 constexpr uint32_t kBsaSmemV = 4 * 32768;       // 2 stages x 32 KB
-constexpr uint32_t kBsaSmemBytes = 6 * 32768 + 1024;  // + alignment slack
+constexpr uint32_t kBsaSmemR = 6 * 32768;       // packed R_b (merge variant), 32 KB
+constexpr uint32_t kBsaSmemBytes = 6 * 32768 + 1024;       // + alignment slack
+constexpr uint32_t kBsaMergeSmemBytes = 7 * 32768 + 1024;
+constexpr uint32_t kRImageBytes = 32768;  // one packed R_b tile (bf16, 128B-swizzled MN-major)
 constexpr int kBsaRowsPerCta = 2 * kTile;
 
 struct BsaParams {
@@ -55,8 +69,19 @@ struct BsaParams {
   int64_t o_row_stride;  // elements between consecutive tokens
   int d_store;           // leading columns of each head row to store
   float* lse;            // optional [H][N]
+  // merge variant only
+  const uint8_t* rimg;   // [nb][H] packed R_b tiles of kRImageBytes
+  const void* g_s;       // [N][H] gate logits
+  const void* g_l;
+  int gate_f32;
+  const float* rms_w;    // [H][d]
+  float eps;
+  void* out;             // [N][H][d]
+  int out_f32;
+  int d;                 // real head dim
 };
 
+template <bool kMerge>
 __global__ void __launch_bounds__(kBsaThreads, 1)
     k_bsa_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkt,
@@ -71,7 +96,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q, bar_kf[2], bar_ke[2], bar_vf[2], bar_ve[2], bar_sf[2], bar_pf[2],
-      bar_of[2];
+      bar_of[2], bar_r;
+  __shared__ float w_sm[128];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -83,6 +109,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(q_full, 1);
+    mbar_init(smem_u32(&bar_r), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bar_kf[i]), 1);
       mbar_init(smem_u32(&bar_ke[i]), 1);
@@ -98,6 +125,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     tmem_alloc(smem_u32(&tmem_slot), 512);
     tmem_relinquish();
   }
+  if (kMerge && threadIdx.x < 128)
+    w_sm[threadIdx.x] = (threadIdx.x < p.d) ? __ldg(p.rms_w + (int64_t)h * p.d + threadIdx.x) : 0.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -106,7 +135,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   // Each role's code sits inside the branch that set its register budget, so
   // no path joins two budgets before the common teardown.
   if (warp >= 8) {
-  regs_dealloc<kBsaRegsProducer>();
+  regs_dealloc<kMerge ? kBsaMergeRegsProducer : kBsaRegsProducer>();
   if (warp == 8) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
@@ -118,6 +147,11 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       tma_load_3d(sQ + 16384, &tq, q_full, 64, h, qs);
       tma_load_3d(sQ + 32768, &tq, q_full, 0, h, qs + kTile);
       tma_load_3d(sQ + 49152, &tq, q_full, 64, h, qs + kTile);
+      if (kMerge) {
+        mbar_arrive_expect_tx(smem_u32(&bar_r), kRImageBytes);
+        bulk_load(base + kBsaSmemR, p.rimg + ((int64_t)b * p.H + h) * kRImageBytes, kRImageBytes,
+                  smem_u32(&bar_r));
+      }
       for (int j = 0; j < nkt; ++j) {
         if (*abort_v) break;
         const int st = j & 1;
@@ -168,6 +202,16 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
           umma_bf16_ts(dO, aP + (uint32_t)(s * 8), sdesc_sw128(sV + (uint32_t)(s * 2048), 16384, 1024),
                        idO, (acc || s > 0) ? 1u : 0u);
       };
+      // o_lin_i = Q_i R_b into the S_i columns (merge variant, after PV_i's last tile)
+      auto readout = [&](int i) {
+        const uint32_t sQi = sQ + (uint32_t)i * 32768u;
+        const uint32_t sR = base + kBsaSmemR;
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          umma_bf16_ss(tmem + (uint32_t)(i * 128),
+                       sdesc_sw128(sQi + (uint32_t)((s >> 2) * 16384 + (s & 3) * 32), 16, 1024),
+                       sdesc_sw128(sR + (uint32_t)(s * 2048), 16384, 1024), idO, s > 0 ? 1u : 0u);
+      };
       bool ok = mbar_wait(q_full, 0) && mbar_wait(smem_u32(&bar_kf[0]), 0);
       if (ok) {
         tc_fence_after();
@@ -186,7 +230,14 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         if (!mbar_wait(smem_u32(&bar_pf[0]), (uint32_t)(j & 1))) { ok = false; break; }
         tc_fence_after();
         pv(0, st, j > 0);
-        if (!more) umma_commit(smem_u32(&bar_of[0]));
+        if (!more) {
+          if (kMerge) {
+            if (!mbar_wait(smem_u32(&bar_r), 0)) { ok = false; break; }
+            tc_fence_after();
+            readout(0);
+          }
+          umma_commit(smem_u32(&bar_of[0]));
+        }
         if (more) {
           if (!mbar_wait(smem_u32(&bar_kf[st1]), ph1)) { ok = false; break; }
           tc_fence_after();
@@ -196,7 +247,10 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         tc_fence_after();
         pv(1, st, j > 0);
         umma_commit(smem_u32(&bar_ve[st]));
-        if (!more) umma_commit(smem_u32(&bar_of[1]));
+        if (!more) {
+          if (kMerge) readout(1);
+          umma_commit(smem_u32(&bar_of[1]));
+        }
         if (more) {
           qk(1, st1);
           umma_commit(smem_u32(&bar_ke[st1]));
@@ -207,7 +261,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     __syncwarp();
   }
   } else {
-    regs_alloc<kBsaRegsSoftmax>();
+    regs_alloc<kMerge ? kBsaMergeRegsSoftmax : kBsaRegsSoftmax>();
     // ---------------------------------------------------- softmax warps --
     const int tile = warp >> 2;             // query tile of this warpgroup
     const int r = threadIdx.x & 127;        // row within the tile == TMEM lane
@@ -297,36 +351,115 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     const int row = qs + tile * kTile + r;
     const bool store = ok && row < q1;
     const float inv = 1.f / l_sum;
-    __nv_bfloat16* dst = p.o + (int64_t)row * p.o_row_stride + (int64_t)h * p.d_store;
-    // the TMEM loads are warp-collective: every thread runs them, only the
-    // stores depend on the row
+    if (!kMerge) {
+      __nv_bfloat16* dst = p.o + (int64_t)row * p.o_row_stride + (int64_t)h * p.d_store;
+      // the TMEM loads are warp-collective: every thread runs them, only the
+      // stores depend on the row
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t o[32];
-      tmem_ld32(tO + (uint32_t)(c * 32), o);
-      tmem_ld_wait(o);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + (uint32_t)(c * 32), o);
+        tmem_ld_wait(o);
+        if (store) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (c * 32 + u * 8 < p.d_store) {
+              uint4 val;
+              val.x = pack_bf16x2(__uint_as_float(o[u * 8 + 0]) * inv, __uint_as_float(o[u * 8 + 1]) * inv);
+              val.y = pack_bf16x2(__uint_as_float(o[u * 8 + 2]) * inv, __uint_as_float(o[u * 8 + 3]) * inv);
+              val.z = pack_bf16x2(__uint_as_float(o[u * 8 + 4]) * inv, __uint_as_float(o[u * 8 + 5]) * inv);
+              val.w = pack_bf16x2(__uint_as_float(o[u * 8 + 6]) * inv, __uint_as_float(o[u * 8 + 7]) * inv);
+              *reinterpret_cast<uint4*>(dst + c * 32 + u * 8) = val;
+            }
+          }
+        }
+      }
+      if (store && p.lse != nullptr)
+        p.lse[(int64_t)h * p.N + row] = (m_use + __log2f(l_sum)) * 0.69314718055994531f;
+    } else {
+      // gated merge of O / l with RMSNorm(o_lin); o_lin sits in the S_i columns
+      const int64_t gi = (int64_t)row * p.H + h;
+      float gs = 0.f, gl = 0.f;
       if (store) {
+        gs = p.gate_f32 ? __ldg(reinterpret_cast<const float*>(p.g_s) + gi)
+                        : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.g_s)[gi]);
+        gl = p.gate_f32 ? __ldg(reinterpret_cast<const float*>(p.g_l) + gi)
+                        : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.g_l)[gi]);
+      }
+      float ss = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (c * 32 + u * 8 < p.d_store) {
-            uint4 val;
-            val.x = pack_bf16x2(__uint_as_float(o[u * 8 + 0]) * inv, __uint_as_float(o[u * 8 + 1]) * inv);
-            val.y = pack_bf16x2(__uint_as_float(o[u * 8 + 2]) * inv, __uint_as_float(o[u * 8 + 3]) * inv);
-            val.z = pack_bf16x2(__uint_as_float(o[u * 8 + 4]) * inv, __uint_as_float(o[u * 8 + 5]) * inv);
-            val.w = pack_bf16x2(__uint_as_float(o[u * 8 + 6]) * inv, __uint_as_float(o[u * 8 + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + c * 32 + u * 8) = val;
+      for (int c = 0; c < 4; ++c) {
+        uint32_t z[32];
+        tmem_ld32(tS + (uint32_t)(c * 32), z);
+        tmem_ld_wait(z);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(z[e]), __uint_as_float(z[e]), ss);
+      }
+      const float a_s = inv / (1.f + __expf(-gs));
+      const float a_l = rsqrtf(ss / (float)p.d + p.eps) / (1.f + __expf(-gl));
+      const int64_t obase = gi * p.d;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32], z[32];
+        tmem_ld32(tO + (uint32_t)(c * 32), o);
+        tmem_ld32(tS + (uint32_t)(c * 32), z);
+        tmem_ld_wait(o);
+        tmem_ld_wait(z);
+        if (store) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c0 = c * 32 + u * 8;
+            if (c0 < p.d) {
+              float y[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                y[e] = a_s * __uint_as_float(o[u * 8 + e]) +
+                       a_l * w_sm[c0 + e] * __uint_as_float(z[u * 8 + e]);
+              if (p.out_f32) {
+                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + obase + c0);
+                dst[0] = make_float4(y[0], y[1], y[2], y[3]);
+                dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+              } else {
+                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + obase + c0) =
+                    make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                               pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+              }
+            }
           }
         }
       }
     }
-    if (store && p.lse != nullptr)
-      p.lse[(int64_t)h * p.N + row] = (m_use + __log2f(l_sum)) * 0.69314718055994531f;
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// R_b = Rfwd + Rbwd (fp32, padded 128 x 128) -> bf16 tile image laid out
+// exactly as the merge variant's shared-memory B operand (128B-swizzled,
+// MN-major: row k of 128 B per 64 value dims, two 16 KB chunks), so the CTA
+// fetches it with one bulk copy. One CTA per (block, head), thread = row.
+__global__ void k_pack_read_states(const float* __restrict__ ra, const float* __restrict__ rb,
+                                   uint8_t* __restrict__ img) {
+  const int64_t bh = blockIdx.x;
+  const int i = threadIdx.x;
+  const float4* a = reinterpret_cast<const float4*>(ra + (bh * 128 + i) * 128);
+  const float4* c4 = reinterpret_cast<const float4*>(rb + (bh * 128 + i) * 128);
+  uint8_t* dst = img + bh * kRImageBytes;
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int q = ch * 16 + u * 2;
+      const float4 x0 = __ldg(a + q), x1 = __ldg(a + q + 1);
+      const float4 y0 = __ldg(c4 + q), y1 = __ldg(c4 + q + 1);
+      *reinterpret_cast<uint4*>(dst + ch * 16384 + sw128_off((uint32_t)i, (uint32_t)u)) =
+          make_uint4(pack_bf16x2(x0.x + y0.x, x0.y + y0.y), pack_bf16x2(x0.z + y0.z, x0.w + y0.w),
+                     pack_bf16x2(x1.x + y1.x, x1.y + y1.y), pack_bf16x2(x1.z + y1.z, x1.w + y1.w));
+    }
   }
 }
 

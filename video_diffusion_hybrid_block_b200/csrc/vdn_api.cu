@@ -84,7 +84,7 @@ struct Plan {
   int dtype;
   int max_qtiles;
   bool staged;  // inputs are narrowed / padded into the workspace
-  size_t o_q, o_k, o_v, o_kt, o_vt, o_osoft, o_C, o_W, o_R, total;
+  size_t o_q, o_k, o_v, o_kt, o_vt, o_osoft, o_C, o_W, o_R, o_Rimg, total;
   const int32_t* off_dev;
 };
 
@@ -136,6 +136,7 @@ int make_plan(const vdn_shape_t* s, Plan* P) {
   P->o_C = o; o += align256(mat);
   P->o_W = o; o += align256(mat);
   P->o_R = o; o += align256((size_t)2 * P->nb * P->H * 128 * 128 * 4);
+  P->o_Rimg = o; o += align256((size_t)P->nb * P->H * kRImageBytes);
   P->total = o;
   return VDN_OK;
 }
@@ -148,8 +149,10 @@ bool set_smem_attrs() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (done[dev]) return true;
-  bool ok = cudaFuncSetAttribute(k_bsa_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  bool ok = cudaFuncSetAttribute(k_bsa_fwd<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kBsaSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_bsa_fwd<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kBsaMergeSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_vda_gram_inv, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kGramSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_vda_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -246,8 +249,18 @@ int launch_vda(const Plan& P, const Acts& a, uint8_t* ws, cudaStream_t st, float
   return VDN_OK;
 }
 
+struct MergeArgs {
+  const void* g_s;
+  const void* g_l;
+  const float* rms_w;
+  void* out;
+};
+
+// Softmax branch; with `merge` set, the readout + gated merge run in its
+// epilogue (R_b packed images at ws + o_Rimg must be ready) and `out` is
+// written instead of o_soft.
 int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int64_t o_row,
-               int d_store, float* lse, cudaStream_t st) {
+               int d_store, float* lse, cudaStream_t st, const MergeArgs* merge) {
   if (P.N == 0) return VDN_OK;
   CUtensorMap tq, tk, tv, tkt, tvt;
   if (!act_map(&tq, a.q, P.N, P, 128, ws + P.o_C) || !act_map(&tk, a.k, P.N, P, 128, ws + P.o_C) ||
@@ -256,6 +269,7 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
       !act_map(&tvt, a.vt, P.T, P, 128, ws + P.o_C))
     return VDN_ERR_CUDA;
   BsaParams bp;
+  memset(&bp, 0, sizeof(bp));
   bp.off = P.off_dev;
   bp.F = P.F;
   bp.T = P.T;
@@ -267,8 +281,21 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
   bp.o_row_stride = o_row;
   bp.d_store = d_store;
   bp.lse = lse;
-  k_bsa_fwd<<<dim3((P.max_qtiles + 1) / 2, P.nb, P.H), kBsaThreads, kBsaSmemBytes, st>>>(
-      tq, tk, tv, tkt, tvt, bp);
+  bp.d = P.d;
+  const dim3 grid((P.max_qtiles + 1) / 2, P.nb, P.H);
+  if (merge == nullptr) {
+    k_bsa_fwd<false><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, bp);
+  } else {
+    bp.rimg = ws + P.o_Rimg;
+    bp.g_s = merge->g_s;
+    bp.g_l = merge->g_l;
+    bp.gate_f32 = (P.dtype == VDN_F32);
+    bp.rms_w = merge->rms_w;
+    bp.eps = P.eps;
+    bp.out = merge->out;
+    bp.out_f32 = (P.dtype == VDN_F32);
+    k_bsa_fwd<true><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, bp);
+  }
   return VDN_OK;
 }
 
@@ -357,14 +384,13 @@ int vdn_hybrid_attn_fwd(const vdn_shape_t* shape, const void* q, const void* k, 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, true, true);
   rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr);
-  if (rc == VDN_OK)
-    rc = launch_bsa(P, a, ws, reinterpret_cast<__nv_bfloat16*>(ws + P.o_osoft),
-                    (int64_t)P.H * kDPad, kDPad, nullptr, st);
-  const float* R = reinterpret_cast<const float*>(ws + P.o_R);
-  if (rc == VDN_OK)
-    rc = launch_merge(P, a.q, R, R + (size_t)P.nb * P.H * 128 * 128, 128,
-                      reinterpret_cast<const __nv_bfloat16*>(ws + P.o_osoft), (int64_t)P.H * kDPad,
-                      kDPad, g_s, g_l, rms_w, out, ws, st);
+  if (rc == VDN_OK) {
+    const float* R = reinterpret_cast<const float*>(ws + P.o_R);
+    k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
+                                                   ws + P.o_Rimg);
+    MergeArgs m{g_s, g_l, rms_w, out};
+    rc = launch_bsa(P, a, ws, nullptr, 0, kDPad, nullptr, st, &m);
+  }
   return finish(rc);
 }
 
@@ -429,7 +455,8 @@ int vdn_bsa_fwd(const vdn_shape_t* shape, const void* q, const void* k, const vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, true, true);
-  rc = launch_bsa(P, a, ws, static_cast<__nv_bfloat16*>(o_soft), (int64_t)P.H * P.d, P.d, lse, st);
+  rc = launch_bsa(P, a, ws, static_cast<__nv_bfloat16*>(o_soft), (int64_t)P.H * P.d, P.d, lse, st,
+                  nullptr);
   return finish(rc);
 }
 
