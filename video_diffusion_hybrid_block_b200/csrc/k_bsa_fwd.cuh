@@ -30,7 +30,11 @@
 // (for a rescale) from then until it hands over P_i(j+1).
 // Online softmax in the exp2 domain with a lazily updated running max: O and
 // the row sum are rescaled only when the tile max exceeds the max in use by
-// more than 8 (a factor 256), which keeps every P <= 256.
+// more than 8 (a factor 256), which keeps every P <= 256. The exp2 work is
+// split between the MUFU unit (3 of 4 column pairs) and a polynomial on the
+// FMA pipe (1 of 4); measured on pages-scale this beats all-MUFU (2.62 vs
+// 2.68 ms) and both 1/8 and 1/2 splits, while packing P with integer ops
+// instead of cvt.rn.bf16x2 was slower in every split.
 //
 // kMerge = true fuses the linear-branch readout and the gated merge into the
 // epilogue: after the last PV_i the MMA thread issues o_lin_i = Q_i R_b into
@@ -79,25 +83,26 @@ struct BsaParams {
   void* out;             // [N][H][d]
   int out_f32;
   int d;                 // real head dim
+  int tma_out;           // out is bf16 [N][H][128]: full tiles leave through a TMA store
 };
 
 template <bool kMerge>
 __global__ void __launch_bounds__(kBsaThreads, 1)
     k_bsa_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkt,
-              const __grid_constant__ CUtensorMap tvt, const BsaParams p) {
+              const __grid_constant__ CUtensorMap tvt, const __grid_constant__ CUtensorMap tout,
+              const BsaParams p) {
   const int pair = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
   int q0, q1;
   block_rows(p.off, p.F, p.bf, b, q0, q1);
   const int qs = q0 + pair * kBsaRowsPerCta;
   if (qs >= q1) return;  // uniform over the CTA, before any resource is taken
-  const KeySegs segs = key_segments(p.off, p.F, p.bf, p.T, b);
-  const int nkt = segs_tiles(segs);
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q, bar_kf[2], bar_ke[2], bar_vf[2], bar_ve[2], bar_sf[2], bar_pf[2],
       bar_of[2], bar_r;
   __shared__ float w_sm[128];
+  __shared__ KeySegs segs;  // key segments of this block, shared by all roles
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -107,6 +112,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   const uint32_t q_full = smem_u32(&bar_q);
 
   if (threadIdx.x == 0) {
+    segs = key_segments(p.off, p.F, p.bf, p.T, b);
     abort_flag = 0;
     mbar_init(q_full, 1);
     mbar_init(smem_u32(&bar_r), 1);
@@ -132,6 +138,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
+  const int nkt = segs_tiles(segs);
   // Each role's code sits inside the branch that set its register budget, so
   // no path joins two budgets before the common teardown.
   if (warp >= 8) {
@@ -333,7 +340,9 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         for (int e = 0; e < 32; ++e) {
           const int c = half * 64 + 2 * e;
           const float2 x = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2);
-          const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          // one pair in four goes to the FMA pipe, the rest to MUFU ex2
+          const float2 pe = ((e & 3) == 3) ? exp2_poly2(x)
+                                           : make_float2(ex2_approx(x.x), ex2_approx(x.y));
           lacc[e & 3] = fadd2(lacc[e & 3], pe);
           pk[e] = pack_bf16x2(pe.x, pe.y);
         }
@@ -345,6 +354,19 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     }
     const float l_sum = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y) +
                         (lacc[2].x + lacc[2].y) + (lacc[3].x + lacc[3].y);
+    // merge variant: fetch this row's gate logits before waiting on the last
+    // MMAs so the load latency overlaps them
+    float gs = 0.f, gl = 0.f;
+    if (kMerge) {
+      const int grow = qs + tile * kTile + r;
+      if (grow < q1) {
+        const int64_t gi = (int64_t)grow * p.H + h;
+        gs = p.gate_f32 ? __ldg(reinterpret_cast<const float*>(p.g_s) + gi)
+                        : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.g_s)[gi]);
+        gl = p.gate_f32 ? __ldg(reinterpret_cast<const float*>(p.g_l) + gi)
+                        : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.g_l)[gi]);
+      }
+    }
     if (ok && !mbar_wait(smem_u32(&bar_of[tile]), 0)) ok = false;
     if (!ok) *abort_v = 1;
     tc_fence_after();
@@ -379,13 +401,6 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     } else {
       // gated merge of O / l with RMSNorm(o_lin); o_lin sits in the S_i columns
       const int64_t gi = (int64_t)row * p.H + h;
-      float gs = 0.f, gl = 0.f;
-      if (store) {
-        gs = p.gate_f32 ? __ldg(reinterpret_cast<const float*>(p.g_s) + gi)
-                        : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.g_s)[gi]);
-        gl = p.gate_f32 ? __ldg(reinterpret_cast<const float*>(p.g_l) + gi)
-                        : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.g_l)[gi]);
-      }
       float ss = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -398,6 +413,10 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       const float a_s = inv / (1.f + __expf(-gs));
       const float a_l = rsqrtf(ss / (float)p.d + p.eps) / (1.f + __expf(-gl));
       const int64_t obase = gi * p.d;
+      // a full tile of a bf16 d=128 output leaves through the (now idle) Q_i
+      // buffer and one TMA store; otherwise each thread stores its row
+      const bool via_tma = p.tma_out && (qs + tile * kTile + kTile <= q1);
+      const uint32_t stage = sQ + (uint32_t)tile * 32768u;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32], z[32];
@@ -405,27 +424,39 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         tmem_ld32(tS + (uint32_t)(c * 32), z);
         tmem_ld_wait(o);
         tmem_ld_wait(z);
-        if (store) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c0 = c * 32 + u * 8;
-            if (c0 < p.d) {
-              float y[8];
+        for (int u = 0; u < 4; ++u) {
+          const int c0 = c * 32 + u * 8;
+          float y[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                y[e] = a_s * __uint_as_float(o[u * 8 + e]) +
-                       a_l * w_sm[c0 + e] * __uint_as_float(z[u * 8 + e]);
-              if (p.out_f32) {
-                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + obase + c0);
-                dst[0] = make_float4(y[0], y[1], y[2], y[3]);
-                dst[1] = make_float4(y[4], y[5], y[6], y[7]);
-              } else {
-                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + obase + c0) =
-                    make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
-                               pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
-              }
+          for (int e = 0; e < 8; ++e)
+            y[e] = a_s * __uint_as_float(o[u * 8 + e]) + a_l * w_sm[c0 + e] * __uint_as_float(z[u * 8 + e]);
+          if (via_tma) {
+            st_shared_v4(stage + (uint32_t)(c0 >> 6) * 16384u + sw128_off((uint32_t)r, (uint32_t)((c0 & 63) >> 3)),
+                         pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                         pack_bf16x2(y[6], y[7]));
+          } else if (store && c0 < p.d) {
+            if (p.out_f32) {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + obase + c0);
+              dst[0] = make_float4(y[0], y[1], y[2], y[3]);
+              dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+            } else {
+              *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + obase + c0) =
+                  make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                             pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
             }
           }
+        }
+      }
+      if (via_tma) {
+        fence_proxy_async_smem();
+        named_barrier_sync(2 + tile, 128);
+        if (r == 0 && ok) {
+          const int row0 = qs + tile * kTile;
+          tma_store_3d(&tout, stage, 0, h, row0);
+          tma_store_3d(&tout, stage + 16384u, 64, h, row0);
+          bulk_commit_group();
+          bulk_wait_all();
         }
       }
     }

@@ -14,16 +14,22 @@
 // k_vda_gram_inv: one CTA per (matrix m, head): m = 0 is the text, m = f is
 //   latent frame f (1 <= f <= F-2; anchors 0 and F-1 are never scanned).
 //   Streams the frame's k, v rows in 64-token tiles (TMA, 2 stages),
-//   L2-normalises k rows in shared memory, accumulates [G | C] = K^T [K | V]
-//   as one M=128 x N=256 bf16 tcgen05 contraction into TMEM, writes C (fp32)
+//   L2-normalises k rows in shared memory, accumulates G = K^T K and
+//   C^T = V^T K as two M=128 x N=128 bf16 tcgen05 contractions into TMEM,
+//   writes C^T (fp32, the layout the scan loads as its X operand)
 //   and then inverts M = lambda I + G in registers with a Gauss-Jordan sweep
 //   (no pivoting: M is symmetric positive definite with eigenvalues
 //   >= lambda) and writes W = M^-1 (fp32).
-// k_vda_scan: one CTA per (direction, head). Step 0 applies the text
-//   (S = W_t C_t), then one step per frame: X = lambda S + C_f,
-//   S = W_f X as a tf32 tcgen05 contraction (W via TMA, X written
-//   transposed by the threads, D in TMEM). States a block reads go to
-//   Rpart[dir][b]; optional per-frame / text outputs are written too.
+// Only frames whose state some block reads are processed: the forward scan
+//   stops at the largest forward read index, the backward scan at the
+//   smallest backward one (the remaining frames always sit inside the window
+//   of every block that could reach them), unless per-frame states are asked
+//   for.
+// k_vda_scan: one CTA per (direction, head, value-column half). Step 0
+//   applies the text (S = W_t C_t), then one step per frame:
+//   X = lambda S + C_f, S = W_f X as a tf32 tcgen05 contraction (W and C_f^T
+//   via TMA, lambda S^T added in shared memory, D in TMEM). States a block
+//   reads go to Rpart[dir][b]; optional per-frame / text outputs too.
 #pragma once
 
 #include "layer_plan.cuh"
@@ -33,18 +39,21 @@ namespace vdn {
 
 // ------------------------------------------------------------ Gram + inverse
 
-constexpr int kGramThreads = 256;
+constexpr int kGramThreads = 512;
 constexpr int kGramTok = 64;                // tokens per tile
+constexpr int kGramStages = 3;
 constexpr uint32_t kGramStage = 4 * 8192;  // k chunk0, k chunk1, v chunk0, v chunk1
-// 2 stages (64 KB); the request is padded so at most two CTAs share an SM
-// (two x 256 TMEM columns).
-constexpr uint32_t kGramSmemBytes = 100 * 1024;
+// 3 stages (96 KB, reused for G once the Grams are done); at most two CTAs
+// share an SM (two x 256 TMEM columns).
+constexpr uint32_t kGramSmemBytes = kGramStages * kGramStage + 1024;
 
 struct GramParams {
   const int32_t* off;  // [F+1] device
   int F, T, H;
+  int fwd_last;        // frames 1..fwd_last feed the forward scan
+  int bwd_first;       // frames bwd_first..F-2 feed the backward scan
   float lambda;
-  float* Cmat;  // [F-1][H][128][128]
+  float* Cmat;  // [F-1][H][128][128], C^T = V^T K_hat (row = value dim)
   float* Wmat;  // [F-1][H][128][128]
 };
 
@@ -52,7 +61,11 @@ __global__ void __launch_bounds__(kGramThreads, 2)
     k_vda_gram_inv(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                    const __grid_constant__ CUtensorMap tkt, const __grid_constant__ CUtensorMap tvt,
                    const GramParams p) {
-  const int m = blockIdx.x, h = blockIdx.y;
+  // blockIdx.x enumerates the text (0), frames 1..fwd_last, then the frames
+  // max(bwd_first, fwd_last+1)..F-2; matrices keep index m = frame.
+  const int h = blockIdx.y;
+  int m = blockIdx.x;
+  if (m > p.fwd_last) m = imax(p.bwd_first, p.fwd_last + 1) + (m - p.fwd_last - 1);
   const bool text = (m == 0);
   const int r0 = text ? 0 : p.off[m];
   const int r1 = text ? p.T : p.off[m + 1];
@@ -62,23 +75,22 @@ __global__ void __launch_bounds__(kGramThreads, 2)
   const CUtensorMap* mv = text ? &tvt : &tv;
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_full[2], bar_empty[2], bar_done;
+  __shared__ uint64_t bar_full[kGramStages], bar_empty[kGramStages], bar_done;
   __shared__ uint32_t tmem_slot;
-  __shared__ float rowbuf[2][128], colbuf[2][128];
+  __shared__ __align__(16) float rowbuf[2][128];
+  __shared__ __align__(16) float colbuf[2][128];
   __shared__ int abort_flag;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t full[2] = {smem_u32(&bar_full[0]), smem_u32(&bar_full[1])};
-  const uint32_t empty[2] = {smem_u32(&bar_empty[0]), smem_u32(&bar_empty[1])};
   const uint32_t done = smem_u32(&bar_done);
   volatile int* abort_v = &abort_flag;
 
   if (tid == 0) {
     abort_flag = 0;
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(full[i], 1);
-      mbar_init(empty[i], 1);
+    for (int i = 0; i < kGramStages; ++i) {
+      mbar_init(smem_u32(&bar_full[i]), 1);
+      mbar_init(smem_u32(&bar_empty[i]), 1);
     }
     mbar_init(done, 1);
     fence_mbar_init();
@@ -94,34 +106,36 @@ __global__ void __launch_bounds__(kGramThreads, 2)
 
   auto load_tile = [&](int i, int st) {
     const uint32_t dst = base + (uint32_t)st * kGramStage;
+    const uint32_t bar = smem_u32(&bar_full[st]);
     const int row = r0 + i * kGramTok;
-    mbar_arrive_expect_tx(full[st], kGramStage);
-    tma_load_3d(dst, mk, full[st], 0, h, row);
-    tma_load_3d(dst + 8192, mk, full[st], 64, h, row);
-    tma_load_3d(dst + 16384, mv, full[st], 0, h, row);
-    tma_load_3d(dst + 24576, mv, full[st], 64, h, row);
+    mbar_arrive_expect_tx(bar, kGramStage);
+    tma_load_3d(dst, mk, bar, 0, h, row);
+    tma_load_3d(dst + 8192, mk, bar, 64, h, row);
+    tma_load_3d(dst + 16384, mv, bar, 0, h, row);
+    tma_load_3d(dst + 24576, mv, bar, 64, h, row);
   };
   if (tid == 0) {
-    for (int i = 0; i < imin(2, ntiles); ++i) load_tile(i, i);
+    for (int i = 0; i < imin(kGramStages - 1, ntiles); ++i) load_tile(i, i);
   }
 
-  const uint32_t idG = idesc_bf16(128, 256, true, true);
+  const uint32_t idG = idesc_bf16(128, 128, true, true);
   bool ok = true;
   for (int i = 0; i < ntiles; ++i) {
-    const int st = i & 1;
-    const uint32_t ph = (i >> 1) & 1;
-    if (*abort_v || !mbar_wait(full[st], ph)) { ok = false; *abort_v = 1; }
+    const int st = i % kGramStages;
+    const uint32_t ph = (uint32_t)((i / kGramStages) & 1);
+    if (*abort_v || !mbar_wait(smem_u32(&bar_full[st]), ph)) { ok = false; *abort_v = 1; }
     __syncthreads();
     if (*abort_v) { ok = false; break; }
-    // L2-normalise k rows (zero rows beyond the frame, and their v rows)
+    // L2-normalise k rows (zero rows beyond the frame, and their v rows):
+    // 8 threads per token row, 16 elements (two 16-byte units) each
     const uint32_t stage = base + (uint32_t)st * kGramStage;
-    const int row = tid >> 2, quarter = tid & 3;
-    const uint32_t chunk = (uint32_t)(quarter >> 1);
-    const uint32_t u0 = (uint32_t)((quarter & 1) * 4);
-    uint4 kv[4];
+    const int row = tid >> 3, part = tid & 7;
+    const uint32_t chunk = (uint32_t)(part >> 2);
+    const uint32_t u0 = (uint32_t)((part & 3) * 2);
+    uint4 kv[2];
     float ss = 0.f;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       kv[u] = ld_shared_v4(stage + chunk * 8192 + sw128_off((uint32_t)row, u0 + u));
       const uint32_t w4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
 #pragma unroll
@@ -132,10 +146,11 @@ __global__ void __launch_bounds__(kGramThreads, 2)
     }
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
     const bool valid = (i * kGramTok + row) < nrows;
     const float sc = valid ? 1.f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const uint32_t w4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
       uint32_t o4[4];
 #pragma unroll
@@ -152,16 +167,25 @@ __global__ void __launch_bounds__(kGramThreads, 2)
       tc_fence_after();
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
-        const uint64_t d = sdesc_sw128(stage + (uint32_t)(s * 2048), 8192, 1024);
-        umma_bf16_ss(tmem, d, d, idG, (i > 0 || s > 0) ? 1u : 0u);
+        // G = K^T K (A = K^T, B = K) and C^T = V^T K (A = V^T, B = K): all
+        // operands MN-major straight from the TMA tiles
+        const uint64_t dk = sdesc_sw128(stage + (uint32_t)(s * 2048), 8192, 1024);
+        const uint64_t dv = sdesc_sw128(stage + 16384u + (uint32_t)(s * 2048), 8192, 1024);
+        const uint32_t acc = (i > 0 || s > 0) ? 1u : 0u;
+        umma_bf16_ss(tmem, dk, dk, idG, acc);
+        umma_bf16_ss(tmem + 128u, dv, dk, idG, acc);
       }
-      umma_commit(empty[st]);
+      umma_commit(smem_u32(&bar_empty[st]));
       if (i == ntiles - 1) umma_commit(done);
-      if (i + 2 < ntiles) {
-        if (!mbar_wait(empty[st], ph)) {
+      // refill the stage the previous tile used (its MMAs are most likely
+      // done already) with the tile two ahead
+      const int nxt = i + kGramStages - 1;
+      if (nxt < ntiles) {
+        const int sp = nxt % kGramStages;
+        if (i > 0 && !mbar_wait(smem_u32(&bar_empty[sp]), (uint32_t)(((i - 1) / kGramStages) & 1))) {
           *abort_v = 1;
         } else {
-          load_tile(i + 2, st);
+          load_tile(nxt, sp);
         }
       }
     }
@@ -171,31 +195,34 @@ __global__ void __launch_bounds__(kGramThreads, 2)
   tc_fence_after();
   __syncthreads();
 
-  // TMEM -> C (global, fp32) and G (shared, fp32, 16-byte units XOR-swizzled)
+  // TMEM -> C^T (global, fp32) and G (shared, fp32, 16-byte units XOR-swizzled).
+  // 16 warps: lane quarter = warp % 4, 64-column group = warp / 4 (groups 0-1
+  // are G, 2-3 are C^T).
   const uint32_t gs = base;  // reuses the (now idle) staging buffers: 64 KB
   {
-    const int wq = warp & 3;
-    const int i = wq * 32 + lane;
-    float* cdst = p.Cmat + (((int64_t)m * p.H + h) * 128 + i) * 128;
+    const int wq = warp & 3, cg = warp >> 2;
+    const int r = wq * 32 + lane;
+    float* cdst = p.Cmat + (((int64_t)m * p.H + h) * 128 + r) * 128 + (cg - 2) * 64;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t r[32];
+    for (int c = 0; c < 2; ++c) {
+      uint32_t v[32];
       if (ntiles > 0) {
-        tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + (warp < 4 ? 0u : 128u) + (uint32_t)(c * 32), r);
-        tmem_ld_wait(r);
+        tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(cg * 64 + c * 32), v);
+        tmem_ld_wait(v);
       } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = 0u;
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
 #pragma unroll
       for (int uu = 0; uu < 8; ++uu) {
-        const int u = c * 8 + uu;
-        if (warp >= 4)
-          reinterpret_cast<uint4*>(cdst)[u] =
-              make_uint4(r[4 * uu], r[4 * uu + 1], r[4 * uu + 2], r[4 * uu + 3]);
-        else
-          st_shared_v4(gs + (uint32_t)i * 512u + (((uint32_t)u ^ (uint32_t)(i & 31)) << 4),
-                       r[4 * uu], r[4 * uu + 1], r[4 * uu + 2], r[4 * uu + 3]);
+        if (cg >= 2) {
+          reinterpret_cast<uint4*>(cdst + c * 32)[uu] =
+              make_uint4(v[4 * uu], v[4 * uu + 1], v[4 * uu + 2], v[4 * uu + 3]);
+        } else {
+          const uint32_t u = (uint32_t)(cg * 16 + c * 8 + uu);  // 16-byte unit of the G row
+          st_shared_v4(gs + (uint32_t)r * 512u + ((u ^ (uint32_t)(r & 31)) << 4), v[4 * uu],
+                       v[4 * uu + 1], v[4 * uu + 2], v[4 * uu + 3]);
+        }
       }
     }
   }
@@ -206,12 +233,13 @@ __global__ void __launch_bounds__(kGramThreads, 2)
     tmem_dealloc(tmem, 256);
   }
 
-  // Gauss-Jordan inverse of M = lambda I + G, 8x8 register tile per thread.
+  // Gauss-Jordan inverse of M = lambda I + G: thread (ty, tx) holds rows
+  // 4ty..4ty+3, columns 8tx..8tx+7 (32 x 16 threads), one barrier per pivot.
   const int ty = tid >> 4, tx = tid & 15;
-  float a[8][8];
+  float a[4][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t R = (uint32_t)(8 * ty + i);
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t R = (uint32_t)(4 * ty + i);
 #pragma unroll
     for (int hlf = 0; hlf < 2; ++hlf) {
       const uint4 v = ld_shared_v4(gs + R * 512u + ((((uint32_t)(2 * tx + hlf)) ^ (R & 31u)) << 4));
@@ -221,49 +249,73 @@ __global__ void __launch_bounds__(kGramThreads, 2)
       a[i][4 * hlf + 3] = __uint_as_float(v.w);
     }
   }
-  if (ty == tx) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a[i][i] += p.lambda;
-  }
-  for (int kb8 = 0; kb8 < 16; ++kb8) {
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const int k = kb8 * 8 + kk;
+    for (int j = 0; j < 8; ++j)
+      if (4 * ty + i == 8 * tx + j) a[i][j] += p.lambda;
+  for (int kb = 0; kb < 32; ++kb) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int k = kb * 4 + kk;      // pivot; its row lives in thread row ty == kb
       const int buf = k & 1;
-      if (ty == kb8) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) rowbuf[buf][8 * tx + j] = a[kk][j];
+      const int cx = k >> 3, cj = k & 7;  // its column lives in thread column tx == cx
+      if (ty == kb) {
+        *reinterpret_cast<float4*>(&rowbuf[buf][8 * tx]) = make_float4(a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
+        *reinterpret_cast<float4*>(&rowbuf[buf][8 * tx + 4]) = make_float4(a[kk][4], a[kk][5], a[kk][6], a[kk][7]);
       }
-      if (tx == kb8) {
+      if (tx == cx) {
+        float c4[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) colbuf[buf][8 * ty + i] = a[i][kk];
+        for (int i = 0; i < 4; ++i) {
+          float v = a[i][0];
+#pragma unroll
+          for (int j = 1; j < 8; ++j) v = (j == cj) ? a[i][j] : v;
+          c4[i] = v;
+        }
+        *reinterpret_cast<float4*>(&colbuf[buf][4 * ty]) = make_float4(c4[0], c4[1], c4[2], c4[3]);
       }
       __syncthreads();
       const float ip = 1.f / rowbuf[buf][k];
-      float rj[8], ci[8];
+      const float4 r0 = *reinterpret_cast<const float4*>(&rowbuf[buf][8 * tx]);
+      const float4 r1 = *reinterpret_cast<const float4*>(&rowbuf[buf][8 * tx + 4]);
+      const float4 c0 = *reinterpret_cast<const float4*>(&colbuf[buf][4 * ty]);
+      const float rj[8] = {r0.x * ip, r0.y * ip, r0.z * ip, r0.w * ip,
+                           r1.x * ip, r1.y * ip, r1.z * ip, r1.w * ip};
+      const float ci[4] = {c0.x, c0.y, c0.z, c0.w};
+      // rank-1 update a -= c r^T / pivot, two columns per instruction
 #pragma unroll
-      for (int j = 0; j < 8; ++j) rj[j] = rowbuf[buf][8 * tx + j] * ip;
+      for (int i = 0; i < 4; ++i) {
+        const float2 nc = make_float2(-ci[i], -ci[i]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ci[i] = colbuf[buf][8 * ty + i];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) a[i][j] = fmaf(-ci[i], rj[j], a[i][j]);
-      if (ty == kb8) {
+        for (int j = 0; j < 8; j += 2) {
+          const float2 upd = ffma2(nc, make_float2(rj[j], rj[j + 1]), make_float2(a[i][j], a[i][j + 1]));
+          a[i][j] = upd.x;
+          a[i][j + 1] = upd.y;
+        }
+      }
+      if (ty == kb) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) a[kk][j] = rj[j];
       }
-      if (tx == kb8) {
+      if (tx == cx) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a[i][kk] = -ci[i] * ip;
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j == cj) a[i][j] = -ci[i] * ip;
       }
-      if (ty == kb8 && tx == kb8) a[kk][kk] = ip;
+      if (ty == kb && tx == cx) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j == cj) a[kk][j] = ip;
+      }
     }
   }
   float* wdst = p.Wmat + ((int64_t)m * p.H + h) * 128 * 128;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float4* rowp = reinterpret_cast<float4*>(wdst + (int64_t)(8 * ty + i) * 128 + 8 * tx);
+  for (int i = 0; i < 4; ++i) {
+    float4* rowp = reinterpret_cast<float4*>(wdst + (int64_t)(4 * ty + i) * 128 + 8 * tx);
     rowp[0] = make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
     rowp[1] = make_float4(a[i][4], a[i][5], a[i][6], a[i][7]);
   }
@@ -272,13 +324,15 @@ __global__ void __launch_bounds__(kGramThreads, 2)
 // --------------------------------------------------------------- scans ----
 
 constexpr int kScanThreads = 128;
-constexpr uint32_t kScanSmemW = 0;          // 2 stages x 64 KB
-constexpr uint32_t kScanSmemX = 2 * 65536;  // X^T, 64 KB
-constexpr uint32_t kScanSmemBytes = 3 * 65536 + 1024;
+constexpr int kScanHalf = 64;                 // value columns of S per CTA
+constexpr uint32_t kScanSmemW = 0;            // 2 stages x 64 KB (W, fp32 K-major)
+constexpr uint32_t kScanSmemX = 2 * 65536;    // 2 stages x 32 KB (X^T half, fp32 K-major)
+constexpr uint32_t kScanSmemBytes = 2 * 65536 + 2 * 32768 + 1024;
 
 struct ScanParams {
-  const float* Cmat;  // [F-1][H][128][128]
   int F, H, bf, nb;
+  int steps_fwd;      // text + frames 1..steps_fwd-1
+  int steps_bwd;      // text + frames F-2 down to F-steps_bwd
   float lambda;
   float* Rpart;       // [2][nb][H][128][128]
   float* text_out;    // optional [H][d][d]
@@ -287,34 +341,35 @@ struct ScanParams {
   int d_out;
 };
 
-__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
-  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(__float_as_uint(v)) : "memory");
-}
-
+// One CTA per (direction, head, half of the value columns): the columns of
+// S evolve independently (S_f = W_f (lambda S_prev + C_f) acts column-wise),
+// so two CTAs split a chain without exchanging anything. Per step the CTA
+// TMA-loads W_f (128 x 128) and its 64 rows of C_f^T into two-stage rings,
+// adds lambda S_prev^T in place (thread i owns key row i of S, TMEM lane i),
+// and runs 16 tf32 MMAs (M128 N64 K8, both operands K-major).
 __global__ void __launch_bounds__(kScanThreads, 1)
-    k_vda_scan(const __grid_constant__ CUtensorMap tw, const ScanParams p) {
-  const int dir = blockIdx.x, h = blockIdx.y;
+    k_vda_scan(const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tct,
+               const ScanParams p) {
+  const int dir = blockIdx.x, h = blockIdx.y, g = blockIdx.z;
   const int F = p.F;
-  const int nsteps = F - 1;
+  const int nsteps = dir == 0 ? p.steps_fwd : p.steps_bwd;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t bar_w[2], bar_mma;
+  __shared__ uint64_t bar_full[2], bar_mma;
   __shared__ uint32_t tmem_slot;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sW[2] = {base + kScanSmemW, base + kScanSmemW + 65536};
-  const uint32_t sX = base + kScanSmemX;
   const int i = threadIdx.x, warp = i >> 5;
-  const uint32_t wfull[2] = {smem_u32(&bar_w[0]), smem_u32(&bar_w[1])};
+  const uint32_t full[2] = {smem_u32(&bar_full[0]), smem_u32(&bar_full[1])};
   const uint32_t mma_bar = smem_u32(&bar_mma);
 
   if (i == 0) {
-    mbar_init(wfull[0], 1);
-    mbar_init(wfull[1], 1);
+    mbar_init(full[0], 1);
+    mbar_init(full[1], 1);
     mbar_init(mma_bar, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&tmem_slot), 128);
+    tmem_alloc(smem_u32(&tmem_slot), 64);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -325,82 +380,70 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 
   auto mat_of = [&](int s) -> int { return (s == 0) ? 0 : (dir == 0 ? s : F - 1 - s); };
   auto idx_of = [&](int s) -> int { return dir == 0 ? s : (s == 0 ? F - 1 : F - 1 - s); };
-  auto load_w = [&](int s, int st) {
+  auto load_step = [&](int s, int st) {
     const int row = (mat_of(s) * p.H + h) * 128;
-    mbar_arrive_expect_tx(wfull[st], 65536);
+    const uint32_t sW = base + kScanSmemW + (uint32_t)st * 65536u;
+    const uint32_t sX = base + kScanSmemX + (uint32_t)st * 32768u;
+    mbar_arrive_expect_tx(full[st], 65536 + 32768);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) tma_load_2d(sW[st] + (uint32_t)(c * 16384), &tw, wfull[st], c * 32, row);
+    for (int c = 0; c < 4; ++c) {
+      tma_load_2d(sW + (uint32_t)(c * 16384), &tw, full[st], c * 32, row);
+      tma_load_2d(sX + (uint32_t)(c * 8192), &tct, full[st], c * 32, row + g * kScanHalf);
+    }
   };
   if (i == 0) {
     tma_prefetch_desc(&tw);
-    load_w(0, 0);
-    if (nsteps > 1) load_w(1, 1);
+    tma_prefetch_desc(&tct);
+    load_step(0, 0);
+    if (nsteps > 1) load_step(1, 1);
   }
 
-  float creg[128];
-  {
-    const float4* src = reinterpret_cast<const float4*>(
-        p.Cmat + (((int64_t)mat_of(0) * p.H + h) * 128 + i) * 128);
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const float4 v = __ldg(src + u);
-      creg[4 * u] = v.x; creg[4 * u + 1] = v.y; creg[4 * u + 2] = v.z; creg[4 * u + 3] = v.w;
-    }
-  }
-  const uint32_t xcol = sX + (uint32_t)(i >> 5) * 16384u;  // k chunk of this thread's column
-  const uint32_t xu = (uint32_t)((i & 31) >> 2), xb = (uint32_t)((i & 3) * 4);
-  const uint32_t idW = idesc_tf32(128, 128, false, false);
+  // element (n, k = i) of the X^T half: chunk i/32, row n, 4-byte slot of unit (i%32)/4
+  const uint32_t xcol = (uint32_t)(i >> 5) * 8192u + (uint32_t)((i & 3) * 4);
+  const uint32_t xu = (uint32_t)((i & 31) >> 2);
+  const uint32_t idW = idesc_tf32(128, kScanHalf, false, false);
   bool ok = true;
 
   for (int s = 0; s < nsteps && ok; ++s) {
-    // X = lambda * S_prev + C, stored transposed (row n, column i) in 128B-swizzled K-major form
+    const int st = s & 1;
+    const uint32_t sW = base + kScanSmemW + (uint32_t)st * 65536u;
+    const uint32_t sX = base + kScanSmemX + (uint32_t)st * 32768u;
+    if (!mbar_wait(full[st], (uint32_t)((s >> 1) & 1))) { ok = false; break; }
+    if (s > 0) {
+      // X^T[n][i] = C^T[n][i] + lambda S_prev[i][n]
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t sv[32];
-      if (s > 0) {
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[32];
         tmem_ld32(tmem + lane_base + (uint32_t)(c * 32), sv);
         tmem_ld_wait(sv);
-      } else {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) sv[jj] = 0u;
-      }
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        const int n = c * 32 + jj;
-        const float x = fmaf(p.lambda, __uint_as_float(sv[jj]), creg[n]);
-        st_shared_f32(xcol + sw128_off((uint32_t)n, xu) + xb, x);
-      }
-    }
-    if (s + 1 < nsteps) {
-      const float4* src = reinterpret_cast<const float4*>(
-          p.Cmat + (((int64_t)mat_of(s + 1) * p.H + h) * 128 + i) * 128);
-#pragma unroll
-      for (int u = 0; u < 32; ++u) {
-        const float4 v = __ldg(src + u);
-        creg[4 * u] = v.x; creg[4 * u + 1] = v.y; creg[4 * u + 2] = v.z; creg[4 * u + 3] = v.w;
+        for (int jj = 0; jj < 32; ++jj) {
+          const uint32_t n = (uint32_t)(c * 32 + jj);
+          const uint32_t addr = sX + xcol + sw128_off(n, xu);
+          float x;
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(x) : "r"(addr) : "memory");
+          x = fmaf(p.lambda, __uint_as_float(sv[jj]), x);
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(x) : "memory");
+        }
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     named_barrier_sync(1, kScanThreads);
     if (i == 0) {
-      const int st = s & 1;
-      if (!mbar_wait(wfull[st], (uint32_t)((s >> 1) & 1))) {
-        ok = false;
-      } else {
-        tc_fence_after();
+      tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const uint32_t ko = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32);
-          umma_tf32_ss(tmem, sdesc_sw128(sW[st] + ko, 16, 1024), sdesc_sw128(sX + ko, 16, 1024),
-                       idW, k > 0 ? 1u : 0u);
-        }
-        umma_commit(mma_bar);
+      for (int k = 0; k < 16; ++k) {
+        const uint32_t ka = (uint32_t)((k >> 2) * 16384 + (k & 3) * 32);
+        const uint32_t kb = (uint32_t)((k >> 2) * 8192 + (k & 3) * 32);
+        umma_tf32_ss(tmem, sdesc_sw128(sW + ka, 16, 1024), sdesc_sw128(sX + kb, 16, 1024), idW,
+                     k > 0 ? 1u : 0u);
       }
+      umma_commit(mma_bar);
     }
     if (!mbar_wait(mma_bar, (uint32_t)(s & 1))) { ok = false; break; }
     tc_fence_after();
-    if (i == 0 && s + 2 < nsteps) load_w(s + 2, s & 1);
+    if (i == 0 && s + 2 < nsteps) load_step(s + 2, st);
 
     // outputs of this state
     const int idx = idx_of(s);
@@ -413,15 +456,16 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     }
     if (want) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
         tmem_ld32(tmem + lane_base + (uint32_t)(c * 32), sv);
         tmem_ld_wait(sv);
+        const int col0 = g * kScanHalf + c * 32;
         for (int b = 0; b < p.nb; ++b) {
           int i_f, i_b;
           block_read_indices(b, F, p.bf, i_f, i_b);
           if ((dir == 0 ? i_f : i_b) != idx) continue;
-          float* dst = p.Rpart + ((((int64_t)dir * p.nb + b) * p.H + h) * 128 + i) * 128 + c * 32;
+          float* dst = p.Rpart + ((((int64_t)dir * p.nb + b) * p.H + h) * 128 + i) * 128 + col0;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             reinterpret_cast<uint4*>(dst)[u] =
@@ -437,7 +481,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             if (outs[o] == nullptr) continue;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
-              if (c * 32 + jj < p.d_out) outs[o][c * 32 + jj] = __uint_as_float(sv[jj]);
+              if (col0 + jj < p.d_out) outs[o][col0 + jj] = __uint_as_float(sv[jj]);
           }
         }
       }
@@ -447,7 +491,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 64);
   }
 }
 

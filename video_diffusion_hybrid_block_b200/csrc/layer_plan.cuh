@@ -58,12 +58,19 @@ struct KeySegs {
   int first_tile[kMaxSegs + 1];
 };
 
+// Appends a segment. The loops run over compile-time indices only, so a
+// KeySegs value can live in registers (no dynamically indexed local array).
 __host__ __device__ inline void segs_push(KeySegs& s, int src, int a, int e) {
   if (e > a) {
-    s.src[s.n] = src;
-    s.start[s.n] = a;
-    s.len[s.n] = e - a;
-    s.first_tile[s.n + 1] = s.first_tile[s.n] + (e - a + kTile - 1) / kTile;
+#pragma unroll
+    for (int q = 0; q < kMaxSegs; ++q) {
+      if (q == s.n) {
+        s.src[q] = src;
+        s.start[q] = a;
+        s.len[q] = e - a;
+        s.first_tile[q + 1] = s.first_tile[q] + (e - a + kTile - 1) / kTile;
+      }
+    }
     s.n++;
   }
 }
@@ -72,6 +79,13 @@ __host__ __device__ inline KeySegs key_segments(const int32_t* off, int F, int b
                                                 int b) {
   KeySegs s;
   s.n = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxSegs; ++q) {
+    s.src[q] = 0;
+    s.start[q] = 0;
+    s.len[q] = 0;
+    s.first_tile[q + 1] = 0;
+  }
   s.first_tile[0] = 0;
   segs_push(s, 1, 0, T);
   int w0, w1;
@@ -80,6 +94,7 @@ __host__ __device__ inline KeySegs key_segments(const int32_t* off, int F, int b
   int ra[3] = {0, w0, F - 1};
   int rb[3] = {0, w1, F - 1};
   int ca = ra[0], cb = rb[0];
+#pragma unroll
   for (int i = 1; i < 3; ++i) {
     if (ra[i] <= cb + 1) {
       cb = imax(cb, rb[i]);
@@ -93,16 +108,30 @@ __host__ __device__ inline KeySegs key_segments(const int32_t* off, int F, int b
   return s;
 }
 
-__host__ __device__ inline int segs_tiles(const KeySegs& s) { return s.first_tile[s.n]; }
+__host__ __device__ inline int segs_tiles(const KeySegs& s) {
+  int t = 0;
+#pragma unroll
+  for (int q = 1; q <= kMaxSegs; ++q)
+    if (q == s.n) t = s.first_tile[q];
+  return t;
+}
 
 // Key tile j of the list: source, first row, number of valid rows (1..128).
 __host__ __device__ inline void segs_tile(const KeySegs& s, int j, int& src, int& row0,
                                           int& valid) {
-  int i = 0;
-  while (i + 1 < s.n && j >= s.first_tile[i + 1]) ++i;
-  src = s.src[i];
-  row0 = s.start[i] + (j - s.first_tile[i]) * kTile;
-  valid = imin(kTile, s.start[i] + s.len[i] - row0);
+  int sel_src = s.src[0], sel_start = s.start[0], sel_len = s.len[0], sel_ft = 0;
+#pragma unroll
+  for (int q = 1; q < kMaxSegs; ++q) {
+    if (q < s.n && j >= s.first_tile[q]) {
+      sel_src = s.src[q];
+      sel_start = s.start[q];
+      sel_len = s.len[q];
+      sel_ft = s.first_tile[q];
+    }
+  }
+  src = sel_src;
+  row0 = sel_start + (j - sel_ft) * kTile;
+  valid = imin(kTile, sel_start + sel_len - row0);
 }
 
 }  // namespace vdn

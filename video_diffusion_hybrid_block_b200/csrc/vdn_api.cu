@@ -52,13 +52,13 @@ bool map_act(CUtensorMap* m, const void* ptr, int64_t rows, int H, int box_rows)
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [rows, 128] fp32 as a 2-D tensor; box {32, 128}.
-bool map_mat(CUtensorMap* m, const void* ptr, int64_t rows) {
+// [rows, 128] fp32 as a 2-D tensor; box {32, box_rows}.
+bool map_mat(CUtensorMap* m, const void* ptr, int64_t rows, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)128, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)128 * 4};
-  cuuint32_t box[2] = {32, 128};
+  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -218,34 +218,54 @@ bool act_map(CUtensorMap* m, const void* ptr, int64_t rows, const Plan& P, int b
 
 int launch_vda(const Plan& P, const Acts& a, uint8_t* ws, cudaStream_t st, float* text_out,
                float* fwd_out, float* bwd_out) {
-  CUtensorMap tk, tv, tkt, tvt, tw;
+  CUtensorMap tk, tv, tkt, tvt, tw, tct;
   if (!act_map(&tk, a.k, P.N, P, 64, ws + P.o_C) || !act_map(&tv, a.v, P.N, P, 64, ws + P.o_C) ||
       !act_map(&tkt, a.kt, P.T, P, 64, ws + P.o_C) ||
       !act_map(&tvt, a.vt, P.T, P, 64, ws + P.o_C) ||
-      !map_mat(&tw, ws + P.o_W, (int64_t)(P.F - 1) * P.H * 128))
+      !map_mat(&tw, ws + P.o_W, (int64_t)(P.F - 1) * P.H * 128, 128) ||
+      !map_mat(&tct, ws + P.o_C, (int64_t)(P.F - 1) * P.H * 128, kScanHalf))
     return VDN_ERR_CUDA;
+  // Frames the read states depend on (all of them when per-frame states are
+  // requested): forward reads go up to fwd_last, backward reads down to bwd_first.
+  int fwd_last = 0, bwd_first = P.F - 1;
+  for (int b = 0; b < P.nb; ++b) {
+    int i_f, i_b;
+    block_read_indices(b, P.F, P.bf, i_f, i_b);
+    fwd_last = imax(fwd_last, i_f);
+    bwd_first = imin(bwd_first, i_b);
+  }
+  if (fwd_out != nullptr || bwd_out != nullptr) {
+    fwd_last = P.F - 2;
+    bwd_first = 1;
+  }
+  const int n_fwd = fwd_last;                                   // frames 1..fwd_last
+  const int n_bwd = imax(0, (P.F - 2) - imax(bwd_first, fwd_last + 1) + 1);
   GramParams gp;
   gp.off = P.off_dev;
   gp.F = P.F;
   gp.T = P.T;
   gp.H = P.H;
+  gp.fwd_last = fwd_last;
+  gp.bwd_first = bwd_first;
   gp.lambda = P.lambda;
   gp.Cmat = reinterpret_cast<float*>(ws + P.o_C);
   gp.Wmat = reinterpret_cast<float*>(ws + P.o_W);
-  k_vda_gram_inv<<<dim3(P.F - 1, P.H), kGramThreads, kGramSmemBytes, st>>>(tk, tv, tkt, tvt, gp);
+  k_vda_gram_inv<<<dim3(1 + n_fwd + n_bwd, P.H), kGramThreads, kGramSmemBytes, st>>>(tk, tv, tkt,
+                                                                                   tvt, gp);
   ScanParams sp;
-  sp.Cmat = gp.Cmat;
   sp.F = P.F;
   sp.H = P.H;
   sp.bf = P.bf;
   sp.nb = P.nb;
+  sp.steps_fwd = 1 + fwd_last;
+  sp.steps_bwd = 1 + (P.F - 1 - bwd_first);
   sp.lambda = P.lambda;
   sp.Rpart = reinterpret_cast<float*>(ws + P.o_R);
   sp.text_out = text_out;
   sp.fwd_out = fwd_out;
   sp.bwd_out = bwd_out;
   sp.d_out = P.d;
-  k_vda_scan<<<dim3(2, P.H), kScanThreads, kScanSmemBytes, st>>>(tw, sp);
+  k_vda_scan<<<dim3(2, P.H, 128 / kScanHalf), kScanThreads, kScanSmemBytes, st>>>(tw, tct, sp);
   return VDN_OK;
 }
 
@@ -262,12 +282,15 @@ struct MergeArgs {
 int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int64_t o_row,
                int d_store, float* lse, cudaStream_t st, const MergeArgs* merge) {
   if (P.N == 0) return VDN_OK;
-  CUtensorMap tq, tk, tv, tkt, tvt;
+  CUtensorMap tq, tk, tv, tkt, tvt, tout;
   if (!act_map(&tq, a.q, P.N, P, 128, ws + P.o_C) || !act_map(&tk, a.k, P.N, P, 128, ws + P.o_C) ||
       !act_map(&tv, a.v, P.N, P, 128, ws + P.o_C) ||
       !act_map(&tkt, a.kt, P.T, P, 128, ws + P.o_C) ||
       !act_map(&tvt, a.vt, P.T, P, 128, ws + P.o_C))
     return VDN_ERR_CUDA;
+  // the merged output leaves by TMA stores when it is bf16 with d = 128
+  const bool tma_out = merge != nullptr && P.dtype == VDN_BF16 && P.d == kDPad;
+  if (!act_map(&tout, tma_out ? merge->out : a.q, P.N, P, 128, ws + P.o_C)) return VDN_ERR_CUDA;
   BsaParams bp;
   memset(&bp, 0, sizeof(bp));
   bp.off = P.off_dev;
@@ -284,7 +307,7 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
   bp.d = P.d;
   const dim3 grid((P.max_qtiles + 1) / 2, P.nb, P.H);
   if (merge == nullptr) {
-    k_bsa_fwd<false><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, bp);
+    k_bsa_fwd<false><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
   } else {
     bp.rimg = ws + P.o_Rimg;
     bp.g_s = merge->g_s;
@@ -294,7 +317,8 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
     bp.eps = P.eps;
     bp.out = merge->out;
     bp.out_f32 = (P.dtype == VDN_F32);
-    k_bsa_fwd<true><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, bp);
+    bp.tma_out = tma_out ? 1 : 0;
+    k_bsa_fwd<true><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
   }
   return VDN_OK;
 }
