@@ -39,7 +39,7 @@ namespace vdn {
 
 // ------------------------------------------------------------ Gram + inverse
 
-constexpr int kGramThreads = 512;
+constexpr int kGramThreads = 256;
 constexpr int kGramTok = 64;                // tokens per tile
 constexpr int kGramStages = 3;
 constexpr uint32_t kGramStage = 4 * 8192;  // k chunk0, k chunk1, v chunk0, v chunk1
@@ -127,15 +127,15 @@ __global__ void __launch_bounds__(kGramThreads, 2)
     __syncthreads();
     if (*abort_v) { ok = false; break; }
     // L2-normalise k rows (zero rows beyond the frame, and their v rows):
-    // 8 threads per token row, 16 elements (two 16-byte units) each
+    // 4 threads per token row, 32 elements (four 16-byte units) each
     const uint32_t stage = base + (uint32_t)st * kGramStage;
-    const int row = tid >> 3, part = tid & 7;
-    const uint32_t chunk = (uint32_t)(part >> 2);
-    const uint32_t u0 = (uint32_t)((part & 3) * 2);
-    uint4 kv[2];
+    const int row = tid >> 2, part = tid & 3;
+    const uint32_t chunk = (uint32_t)(part >> 1);
+    const uint32_t u0 = (uint32_t)((part & 1) * 4);
+    uint4 kv[4];
     float ss = 0.f;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < 4; ++u) {
       kv[u] = ld_shared_v4(stage + chunk * 8192 + sw128_off((uint32_t)row, u0 + u));
       const uint32_t w4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
 #pragma unroll
@@ -146,11 +146,10 @@ __global__ void __launch_bounds__(kGramThreads, 2)
     }
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
     const bool valid = (i * kGramTok + row) < nrows;
     const float sc = valid ? 1.f / fmaxf(sqrtf(ss), 1e-12f) : 0.f;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < 4; ++u) {
       const uint32_t w4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
       uint32_t o4[4];
 #pragma unroll
@@ -195,19 +194,18 @@ __global__ void __launch_bounds__(kGramThreads, 2)
   tc_fence_after();
   __syncthreads();
 
-  // TMEM -> C^T (global, fp32) and G (shared, fp32, 16-byte units XOR-swizzled).
-  // 16 warps: lane quarter = warp % 4, 64-column group = warp / 4 (groups 0-1
-  // are G, 2-3 are C^T).
+  // TMEM -> C^T (global, fp32) and G (shared, fp32, 16-byte units XOR-swizzled):
+  // lane quarter = warp % 4; warps 0-3 read G, warps 4-7 read C^T.
   const uint32_t gs = base;  // reuses the (now idle) staging buffers: 64 KB
   {
-    const int wq = warp & 3, cg = warp >> 2;
+    const int wq = warp & 3;
     const int r = wq * 32 + lane;
-    float* cdst = p.Cmat + (((int64_t)m * p.H + h) * 128 + r) * 128 + (cg - 2) * 64;
+    float* cdst = p.Cmat + (((int64_t)m * p.H + h) * 128 + r) * 128;
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < 4; ++c) {
       uint32_t v[32];
       if (ntiles > 0) {
-        tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(cg * 64 + c * 32), v);
+        tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + (warp < 4 ? 0u : 128u) + (uint32_t)(c * 32), v);
         tmem_ld_wait(v);
       } else {
 #pragma unroll
@@ -215,14 +213,13 @@ __global__ void __launch_bounds__(kGramThreads, 2)
       }
 #pragma unroll
       for (int uu = 0; uu < 8; ++uu) {
-        if (cg >= 2) {
-          reinterpret_cast<uint4*>(cdst + c * 32)[uu] =
+        const int u = c * 8 + uu;
+        if (warp >= 4)
+          reinterpret_cast<uint4*>(cdst)[u] =
               make_uint4(v[4 * uu], v[4 * uu + 1], v[4 * uu + 2], v[4 * uu + 3]);
-        } else {
-          const uint32_t u = (uint32_t)(cg * 16 + c * 8 + uu);  // 16-byte unit of the G row
-          st_shared_v4(gs + (uint32_t)r * 512u + ((u ^ (uint32_t)(r & 31)) << 4), v[4 * uu],
-                       v[4 * uu + 1], v[4 * uu + 2], v[4 * uu + 3]);
-        }
+        else
+          st_shared_v4(gs + (uint32_t)r * 512u + (((uint32_t)u ^ (uint32_t)(r & 31)) << 4),
+                       v[4 * uu], v[4 * uu + 1], v[4 * uu + 2], v[4 * uu + 3]);
       }
     }
   }
@@ -233,13 +230,13 @@ __global__ void __launch_bounds__(kGramThreads, 2)
     tmem_dealloc(tmem, 256);
   }
 
-  // Gauss-Jordan inverse of M = lambda I + G: thread (ty, tx) holds rows
-  // 4ty..4ty+3, columns 8tx..8tx+7 (32 x 16 threads), one barrier per pivot.
+  // Gauss-Jordan inverse of M = lambda I + G: thread (ty, tx) holds the 8 x 8
+  // tile rows 8ty.., columns 8tx.. (16 x 16 threads), one barrier per pivot.
   const int ty = tid >> 4, tx = tid & 15;
-  float a[4][8];
+  float a[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t R = (uint32_t)(4 * ty + i);
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t R = (uint32_t)(8 * ty + i);
 #pragma unroll
     for (int hlf = 0; hlf < 2; ++hlf) {
       const uint4 v = ld_shared_v4(gs + R * 512u + ((((uint32_t)(2 * tx + hlf)) ^ (R & 31u)) << 4));
@@ -249,43 +246,35 @@ __global__ void __launch_bounds__(kGramThreads, 2)
       a[i][4 * hlf + 3] = __uint_as_float(v.w);
     }
   }
+  if (ty == tx) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i) a[i][i] += p.lambda;
+  }
+  for (int kb8 = 0; kb8 < 16; ++kb8) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (4 * ty + i == 8 * tx + j) a[i][j] += p.lambda;
-  for (int kb = 0; kb < 32; ++kb) {
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const int k = kb * 4 + kk;      // pivot; its row lives in thread row ty == kb
+    for (int kk = 0; kk < 8; ++kk) {
+      const int k = kb8 * 8 + kk;
       const int buf = k & 1;
-      const int cx = k >> 3, cj = k & 7;  // its column lives in thread column tx == cx
-      if (ty == kb) {
+      if (ty == kb8) {
         *reinterpret_cast<float4*>(&rowbuf[buf][8 * tx]) = make_float4(a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
         *reinterpret_cast<float4*>(&rowbuf[buf][8 * tx + 4]) = make_float4(a[kk][4], a[kk][5], a[kk][6], a[kk][7]);
       }
-      if (tx == cx) {
-        float c4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float v = a[i][0];
-#pragma unroll
-          for (int j = 1; j < 8; ++j) v = (j == cj) ? a[i][j] : v;
-          c4[i] = v;
-        }
-        *reinterpret_cast<float4*>(&colbuf[buf][4 * ty]) = make_float4(c4[0], c4[1], c4[2], c4[3]);
+      if (tx == kb8) {
+        *reinterpret_cast<float4*>(&colbuf[buf][8 * ty]) = make_float4(a[0][kk], a[1][kk], a[2][kk], a[3][kk]);
+        *reinterpret_cast<float4*>(&colbuf[buf][8 * ty + 4]) = make_float4(a[4][kk], a[5][kk], a[6][kk], a[7][kk]);
       }
       __syncthreads();
       const float ip = 1.f / rowbuf[buf][k];
       const float4 r0 = *reinterpret_cast<const float4*>(&rowbuf[buf][8 * tx]);
       const float4 r1 = *reinterpret_cast<const float4*>(&rowbuf[buf][8 * tx + 4]);
-      const float4 c0 = *reinterpret_cast<const float4*>(&colbuf[buf][4 * ty]);
+      const float4 c0 = *reinterpret_cast<const float4*>(&colbuf[buf][8 * ty]);
+      const float4 c1 = *reinterpret_cast<const float4*>(&colbuf[buf][8 * ty + 4]);
       const float rj[8] = {r0.x * ip, r0.y * ip, r0.z * ip, r0.w * ip,
                            r1.x * ip, r1.y * ip, r1.z * ip, r1.w * ip};
-      const float ci[4] = {c0.x, c0.y, c0.z, c0.w};
+      const float ci[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
       // rank-1 update a -= c r^T / pivot, two columns per instruction
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 8; ++i) {
         const float2 nc = make_float2(-ci[i], -ci[i]);
 #pragma unroll
         for (int j = 0; j < 8; j += 2) {
@@ -294,28 +283,21 @@ __global__ void __launch_bounds__(kGramThreads, 2)
           a[i][j + 1] = upd.y;
         }
       }
-      if (ty == kb) {
+      if (ty == kb8) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) a[kk][j] = rj[j];
       }
-      if (tx == cx) {
+      if (tx == kb8) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j == cj) a[i][j] = -ci[i] * ip;
+        for (int i = 0; i < 8; ++i) a[i][kk] = -ci[i] * ip;
       }
-      if (ty == kb && tx == cx) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j == cj) a[kk][j] = ip;
-      }
+      if (ty == kb8 && tx == kb8) a[kk][kk] = ip;
     }
   }
   float* wdst = p.Wmat + ((int64_t)m * p.H + h) * 128 * 128;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float4* rowp = reinterpret_cast<float4*>(wdst + (int64_t)(4 * ty + i) * 128 + 8 * tx);
+  for (int i = 0; i < 8; ++i) {
+    float4* rowp = reinterpret_cast<float4*>(wdst + (int64_t)(8 * ty + i) * 128 + 8 * tx);
     rowp[0] = make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
     rowp[1] = make_float4(a[i][4], a[i][5], a[i][6], a[i][7]);
   }
