@@ -136,6 +136,23 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def max_over_ranks(dist, x: float, device) -> float:
+    """The largest of the ranks' values (timing is the max over ranks); dist
+    is torch.distributed or None for a single process. Every rank calls it at
+    the same point."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, flop_per_replica: float, ms: float) -> float:
+    """TFLOP/s of N independent replicas finishing in the max-over-ranks time."""
+    return world * flop_per_replica / (ms * 1e-3) / 1e12
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -192,13 +209,6 @@ def run_cuda(args) -> None:
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # ---- device-resident timing of the whole layer
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
@@ -208,7 +218,7 @@ def run_cuda(args) -> None:
             step()
         e1.record(stream)
         barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    ms = max_over_ranks(dist, e0.elapsed_time(e1) / args.steps, "cuda")
     clocks = clk.summary()
     launches_per_step = 4 + (0 if shape.d == 128 else 5)
 
@@ -229,7 +239,7 @@ def run_cuda(args) -> None:
         bsa()
     b1.record(stream)
     barrier()
-    bsa_ms = max_over_ranks(b0.elapsed_time(b1) / nb_launch)
+    bsa_ms = max_over_ranks(dist, b0.elapsed_time(b1) / nb_launch, "cuda")
 
     # ---- end to end through the C ABI with host buffers (H2D + layer + D2H)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -249,11 +259,11 @@ def run_cuda(args) -> None:
         e2e_step()
     g1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
+    e2e_ms = max_over_ranks(dist, g0.elapsed_time(g1) / args.steps, "cuda")
 
     peaks = load_peaks()
     achieved = fl["softmax"] / (bsa_ms * 1e-3) / 1e12
-    value = world * fl["total"] / (ms * 1e-3) / 1e12
+    value = whole_job_value(world, fl["total"], ms)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -277,7 +287,7 @@ def run_cuda(args) -> None:
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} bf16 burst",
                      "launch_ms": round(bsa_ms, 4), "traffic": recorded_traffic()},
-        "e2e": {"value": round(world * fl["total"] / (e2e_ms * 1e-3) / 1e12, 2),
+        "e2e": {"value": round(whole_job_value(world, fl["total"], e2e_ms), 2),
                 "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
