@@ -233,8 +233,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         const int st1 = (j + 1) & 1;
         const uint32_t ph1 = ((j + 1) >> 1) & 1;
         const bool more = j + 1 < nkt;
-        if (!mbar_wait(smem_u32(&bar_vf[st]), ph)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&bar_pf[0]), (uint32_t)(j & 1))) { ok = false; break; }
+        if (!mbar_wait_spin(smem_u32(&bar_vf[st]), ph)) { ok = false; break; }
+        if (!mbar_wait_spin(smem_u32(&bar_pf[0]), (uint32_t)(j & 1))) { ok = false; break; }
         tc_fence_after();
         pv(0, st, j > 0);
         if (!more) {
@@ -246,11 +246,11 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
           umma_commit(smem_u32(&bar_of[0]));
         }
         if (more) {
-          if (!mbar_wait(smem_u32(&bar_kf[st1]), ph1)) { ok = false; break; }
+          if (!mbar_wait_spin(smem_u32(&bar_kf[st1]), ph1)) { ok = false; break; }
           tc_fence_after();
           qk(0, st1);
         }
-        if (!mbar_wait(smem_u32(&bar_pf[1]), (uint32_t)(j & 1))) { ok = false; break; }
+        if (!mbar_wait_spin(smem_u32(&bar_pf[1]), (uint32_t)(j & 1))) { ok = false; break; }
         tc_fence_after();
         pv(1, st, j > 0);
         umma_commit(smem_u32(&bar_ve[st]));
@@ -296,12 +296,20 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (c >= valid) s[c] = __float_as_uint(-INFINITY);
       }
-      // tile row max of the raw scores (scale > 0 keeps the order)
-      float mx = fmax3(__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]));
+      // tile row max of the raw scores (scale > 0 keeps the order); eight
+      // independent chains of 3-input maxes, then a small tree
+      float mq[8];
 #pragma unroll
-      for (int c = 3; c < 127; c += 2)
-        mx = fmax3(mx, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-      mx = fmaxf(mx, __uint_as_float(s[127]));
+      for (int a = 0; a < 8; ++a)
+        mq[a] = fmax3(__uint_as_float(s[a]), __uint_as_float(s[a + 8]), __uint_as_float(s[a + 16]));
+#pragma unroll
+      for (int c = 24; c < 120; c += 16)
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+          mq[a] = fmax3(mq[a], __uint_as_float(s[c + a]), __uint_as_float(s[c + a + 8]));
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mq[a] = fmaxf(mq[a], __uint_as_float(s[120 + a]));
+      const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(fmax3(mq[3], mq[4], mq[5]), mq[6], mq[7]));
       const float m_tile = mx * scale;
       if (j == 0) {
         m_use = m_tile;
