@@ -32,7 +32,7 @@ METRIC = "hybrid-attn layer fwd ms and TFLOP/s (frac. of bf16 peak), 1×B200"
 WORKLOAD = "pages-scale"
 WORKLOAD_DESC = ("pages-scale single layer: F=15 latent frames (3 blocks of 5), 24x42=1008 "
                  "tokens/frame (15120 video tokens), T=256 text tokens, H=32, d=128, bf16")
-L2_NOTE = "inputs q,k,v,o_soft 4x124 MB > 126 MB L2; no flush between steps"
+L2_BYTES = 126 * 2 ** 20
 
 
 def layer_flops(inp: dict, soft_pairs: np.ndarray) -> dict:
@@ -50,6 +50,21 @@ def layer_flops(inp: dict, soft_pairs: np.ndarray) -> dict:
     solves = (F - 1) * H * (2.0 * d ** 3 + 4.0 * d ** 3)
     return dict(softmax=softmax, vda=grams + readout + solves,
                 total=softmax + grams + readout + solves)
+
+
+def workload_desc(name: str) -> str:
+    if name == WORKLOAD:
+        return WORKLOAD_DESC
+    import vdn_synth as S
+    c = S.CONFIGS[name]
+    return (f"{name}: F={c['F']} latent frames, {c['grid'][0]}x{c['grid'][1]} tokens/frame, "
+            f"T={c['T']}, H={c['H']}, d={c['d']}, {c['dtype']}")
+
+
+def l2_note(input_bytes: int) -> str:
+    if input_bytes > L2_BYTES:
+        return f"inputs {input_bytes / 2 ** 20:.0f} MiB > 126 MB L2; no flush between steps"
+    return "inputs fit in the 126 MB L2: warm-cache figure, no flush between steps"
 
 
 def load_peaks() -> dict:
@@ -175,14 +190,14 @@ def run_cuda(args) -> None:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    inp = S.make_inputs(WORKLOAD, seed=0)
-    dt = torch.bfloat16
+    inp = S.make_inputs(args.workload, seed=0)
+    dt = torch.bfloat16 if inp["dtype"] == "bf16" else torch.float32
     host = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to(dt).pin_memory()
             for k in ("q", "k", "v", "kt", "vt", "g_s", "g_l")}
     dev = {k: t.to("cuda", non_blocking=False) for k, t in host.items()}
     rms_w = torch.from_numpy(inp["rms_w"]).cuda()
     shape = V.Shape(inp["off"], inp["T"], inp["H"], inp["d"], inp["block_frames"], inp["lam"],
-                    inp["eps"], V.VDN_BF16)
+                    inp["eps"], V.VDN_BF16 if inp["dtype"] == "bf16" else V.VDN_F32)
     ws = V.alloc_workspace(shape)
     out = torch.empty_like(dev["q"])
     out_host = torch.empty(out.shape, dtype=dt).pin_memory()
@@ -223,7 +238,7 @@ def run_cuda(args) -> None:
     launches_per_step = 4 + (0 if shape.d == 128 else 5)
 
     # ---- dominant kernel alone (softmax branch), CUDA events on its stream
-    o_soft = torch.empty(dev["q"].shape, dtype=dt, device="cuda")
+    o_soft = torch.empty(dev["q"].shape, dtype=torch.bfloat16, device="cuda")
 
     def bsa():
         V.vdn_bsa_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"], o_soft, None,
@@ -277,23 +292,25 @@ def run_cuda(args) -> None:
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESC, "F": inp["F"], "tokens_per_frame": 1008,
+        "config": {"workload": workload_desc(args.workload), "F": inp["F"],
+                   "tokens_per_frame": int(inp["N"] // inp["F"]),
                    "N": inp["N"], "T": inp["T"], "H": inp["H"], "d": inp["d"],
                    "layer_tflop": round(fl["total"] / 1e12, 4),
                    "softmax_tflop": round(fl["softmax"] / 1e12, 4),
-                   "parallelism": f"replicas x{world}", "l2": L2_NOTE},
+                   "parallelism": f"replicas x{world}", "l2": l2_note(h2d)},
         "roofline": {"kernel": "k_bsa_fwd", "bound": "tensor", "achieved": round(achieved, 1),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} bf16 burst",
-                     "launch_ms": round(bsa_ms, 4), "traffic": recorded_traffic()},
+                     "launch_ms": round(bsa_ms, 4),
+                     "traffic": recorded_traffic() if args.workload == WORKLOAD else None},
         "e2e": {"value": round(whole_job_value(world, fl["total"], e2e_ms), 2),
                 "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
         line["cpu_baseline"] = cpu_baseline(inp, fl, args.cpu_heads)
     if dist is not None:
         dist.barrier()
@@ -420,7 +437,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["layer", "bsa", "vda"],
                     help="only run launches of one entry point (for ncu captures)")
-    ap.add_argument("--workload", default=WORKLOAD, help="workload for --profile")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="workload name (vdn_synth.CONFIGS); the default is the headline one")
     ap.add_argument("--heads", type=int, default=0, help="override head count for --profile")
     args = ap.parse_args()
     if args.profile:
