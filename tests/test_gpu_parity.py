@@ -32,11 +32,25 @@ def _edge_cases():
     ]
 
 
+def _max_jump_case():
+    """Keys scaled by 2^(f//2) per frame (exact in bf16): row maxima of the
+    scores grow by far more than 8 (log2 units) between key tiles, which
+    makes the softmax kernel raise its running max and redo tiles."""
+    inp = S.make_inputs_from(12, [150] * 12, 40, 2, 128, "bf16", seed=8)
+    k = inp["k"].copy()
+    for f in range(12):
+        k[inp["off"][f]:inp["off"][f + 1]] *= 2.0 ** (f // 2)
+    inp["k"] = k
+    return inp
+
+
 def _edge(name):
+    if name == "max-jump":
+        return _max_jump_case()
     return dict(_edge_cases())[name]
 
 
-EDGE = [n for n, _ in _edge_cases()]
+EDGE = [n for n, _ in _edge_cases()] + ["max-jump"]
 
 
 def _cases(name):
