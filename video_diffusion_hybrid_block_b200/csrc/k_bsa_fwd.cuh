@@ -10,7 +10,11 @@
 // head. Key tiles are enumerated from the block's key segments
 // (layer_plan.cuh), so tiles outside the allowed set are never loaded; only
 // the ragged last tile of each segment is masked column-wise. Both query
-// tiles share every K/V tile. Warp roles (384 threads, 3 warpgroups):
+// tiles share every K/V tile. Grid (query-row pairs, heads, blocks): blocks
+// sit on z, which is dispatched last, and are visited interior-first
+// (block_in_visit_order), so the CTAs with the most key tiles start first and
+// the tail of the grid is made of short ones. Warp roles (384 threads, 3
+// warpgroups):
 //   warps 0-3  softmax of query tile 0 (thread r owns row r = TMEM lane r)
 //   warps 4-7  softmax of query tile 1
 //   warp 8     TMA producer: Q0, Q1 once, then K and V tiles (2-stage rings)
@@ -92,7 +96,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkt,
               const __grid_constant__ CUtensorMap tvt, const __grid_constant__ CUtensorMap tout,
               const BsaParams p) {
-  const int pair = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
+  const int pair = blockIdx.x, h = blockIdx.y;
+  const int b = block_in_visit_order(blockIdx.z, num_blocks(p.F, p.bf));
   int q0, q1;
   block_rows(p.off, p.F, p.bf, b, q0, q1);
   const int qs = q0 + pair * kBsaRowsPerCta;

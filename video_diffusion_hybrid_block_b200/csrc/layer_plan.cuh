@@ -41,6 +41,15 @@ __host__ __device__ inline void block_read_indices(int b, int F, int bf, int& i_
   i_bwd = imin(w1 + 1, F - 1);
 }
 
+// Order in which the softmax kernel's CTAs visit blocks: interior blocks
+// (three blocks of window, the most key tiles) before the two edge blocks, so
+// the last CTAs to start are the short ones (longest-first list scheduling).
+__host__ __device__ inline int block_in_visit_order(int z, int nb) {
+  if (nb <= 2) return z;
+  if (z < nb - 2) return z + 1;
+  return z == nb - 2 ? 0 : nb - 1;
+}
+
 // Query rows of block b: [q0, q1).
 __host__ __device__ inline void block_rows(const int32_t* off, int F, int bf, int b, int& q0,
                                            int& q1) {
