@@ -158,6 +158,16 @@ int vdn_vda_scan_noalloc(const vdn_shape_t* shape, const void* k, const void* v,
                          float* text_state, float* fwd_states, float* bwd_states,
                          void* stream);
 
+/* Check of the library's failure detection (no paper counterpart). Launches
+ * one CTA on `stream` that holds `tmem_cols` tensor-memory columns (0, or a
+ * power of two from 32 to 512), waits on a shared-memory barrier phase that
+ * nothing completes through the same bounded wait the kernels use, gives up
+ * after limit_ns nanoseconds (1 <= limit_ns <= 1e9), frees the columns and
+ * returns. Returns VDN_OK once launched (VDN_ERR_INVALID_ARG before any
+ * launch for out-of-range arguments); vdn_get_device_error() then reports
+ * VDN_ERR_DEVICE_TIMEOUT, and the device stays usable. */
+int vdn_selftest_wait_timeout(int64_t limit_ns, int tmem_cols, void* stream);
+
 /* Synchronises the current device, returns VDN_OK or the first device-side
  * error recorded since the last call (VDN_ERR_DEVICE_TIMEOUT for an expired
  * bounded wait), and clears it. */

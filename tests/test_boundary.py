@@ -143,3 +143,10 @@ def test_binding_raises_on_error(lib):
         V.vdn_hybrid_attn_fwd(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
                               stream=0, ws_bytes=1 << 40)
     assert e.value.code == B.VDN_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("limit_ns,cols", [(0, 0), (-5, 0), (1_000_000_001, 0), (1000, 48),
+                                           (1000, 16), (1000, 1024), (1000, -32)])
+def test_selftest_wait_timeout_rejects_bad_arguments(lib, limit_ns, cols):
+    # out-of-range limits or TMEM column counts fail before any launch
+    assert lib.vdn_selftest_wait_timeout(limit_ns, cols, None) == -1

@@ -29,6 +29,8 @@ def _edge_cases():
                                           128, "bf16", seed=4)),
         ("d64-f32", S.make_inputs_from(16, [33] * 16, 12, 3, 64, "f32", seed=5)),
         ("one-token-frames", S.make_inputs_from(23, [1] * 23, 3, 2, 128, "bf16", seed=6)),
+        # no video token at all: the layer writes nothing, the read states are 2 S_text
+        ("empty-video", S.make_inputs_from(7, [0] * 7, 5, 2, 64, "bf16", seed=10)),
     ]
 
 
@@ -44,13 +46,22 @@ def _max_jump_case():
     return inp
 
 
+def _max_frames_case():
+    """The largest frame count the boundary accepts (F = 4096, 820 blocks),
+    frames of 0 to 3 tokens: 4090-step scans in both directions."""
+    sizes = np.random.default_rng(11).integers(0, 4, size=4096)
+    return S.make_inputs_from(4096, sizes, 4, 1, 32, "bf16", seed=9)
+
+
 def _edge(name):
     if name == "max-jump":
         return _max_jump_case()
+    if name == "F4096":
+        return _max_frames_case()
     return dict(_edge_cases())[name]
 
 
-EDGE = [n for n, _ in _edge_cases()] + ["max-jump"]
+EDGE = [n for n, _ in _edge_cases()] + ["max-jump", "F4096"]
 
 
 def _cases(name):

@@ -60,6 +60,7 @@ _SIGS = {
     "vdn_bsa_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
     "vdn_pair_audit": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t), _P, _P, _P]),
     "vdn_vda_scan_noalloc": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 8 + [_P]),
+    "vdn_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int, _P]),
     "vdn_get_device_error": (ctypes.c_int, []),
     "vdn_error_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -203,6 +204,13 @@ def vdn_pair_audit(shape: Shape, soft_pairs, lin_pairs, stream=None):
                                        _stream(stream))
     _check(rc, "vdn_pair_audit")
     return soft_pairs, lin_pairs
+
+
+def vdn_selftest_wait_timeout(limit_ns: int, tmem_cols: int = 0, stream=None):
+    """Launches the bounded-wait failure check (see include/vdn.h); the
+    timeout is then reported by vdn_get_device_error()."""
+    rc = load_library().vdn_selftest_wait_timeout(int(limit_ns), int(tmem_cols), _stream(stream))
+    _check(rc, "vdn_selftest_wait_timeout")
 
 
 def vdn_get_device_error() -> int:

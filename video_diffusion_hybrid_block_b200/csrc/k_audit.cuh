@@ -3,10 +3,12 @@
 // softmax kernel visits (same key_segments / segs_tile enumeration, same
 // valid-row and valid-column masks), and the pairs folded into the linear
 // read states (same block_read_indices the scans use). Integer counts, so the
-// comparison with the oracle's pair classes is exact.
+// comparison with the oracle's pair classes is exact. Also the check of the
+// bounded-wait failure path (k_selftest_wait_timeout).
 #pragma once
 
 #include "layer_plan.cuh"
+#include "sm100_ptx.cuh"
 
 namespace vdn {
 
@@ -58,6 +60,34 @@ __global__ void k_pair_audit_lin(const int32_t* off, int F, int bf, unsigned lon
     // forward state i_f holds frames 1..i_f, backward state i_b frames i_b..F-2
     const bool in = (g >= 1 && g <= i_f) || (g >= i_b && g <= F - 2);
     lin[(int64_t)fq * F + g] = in ? (unsigned long long)(nq * (off[g + 1] - off[g])) : 0ull;
+  }
+}
+
+// Failure-path check of the bounded waits: one CTA (optionally holding TMEM)
+// waits on an mbarrier phase that nothing completes, through the same
+// routine the kernels use, gives up after limit_ns (recording
+// kDevErrWaitTimeout), frees its TMEM and returns, leaving the context usable.
+__global__ void k_selftest_wait_timeout(uint64_t limit_ns, int tmem_cols) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t slot;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  if (tmem_cols > 0 && warp == 0) {
+    tmem_alloc(smem_u32(&slot), (uint32_t)tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) (void)mbar_wait_limit(smem_u32(&bar), 0u, limit_ns);
+  tc_fence_before();
+  __syncthreads();
+  if (tmem_cols > 0 && warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(slot, (uint32_t)tmem_cols);
   }
 }
 

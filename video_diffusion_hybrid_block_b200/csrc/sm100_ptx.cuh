@@ -75,17 +75,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed. Returns false
-// (and records kDevErrWaitTimeout) if it has not after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// (and records kDevErrWaitTimeout) if it has not after limit_ns.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+    if ((i & 31u) == 0 && global_timer_ns() - t0 > limit_ns) {
       record_device_error(kDevErrWaitTimeout);
       return false;
     }
   }
+}
+
+// The kernels' wait: bounded by kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  return mbar_wait_limit(bar, parity, kWaitLimitNs);
 }
 
 // Non-blocking probe of a phase (no suspend): lower wake-up latency than

@@ -502,6 +502,16 @@ int vdn_pair_audit(const vdn_shape_t* shape, int64_t* soft_pairs, int64_t* lin_p
   return finish(VDN_OK);
 }
 
+int vdn_selftest_wait_timeout(int64_t limit_ns, int tmem_cols, void* stream) {
+  if (limit_ns < 1 || limit_ns > 1000000000) return VDN_ERR_INVALID_ARG;
+  if (!(tmem_cols == 0 || tmem_cols == 32 || tmem_cols == 64 || tmem_cols == 128 ||
+        tmem_cols == 256 || tmem_cols == 512))
+    return VDN_ERR_INVALID_ARG;
+  vdn::k_selftest_wait_timeout<<<1, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      (uint64_t)limit_ns, tmem_cols);
+  return cudaGetLastError() == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
 int vdn_get_device_error(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return VDN_ERR_CUDA;
   int v = 0;
