@@ -298,8 +298,11 @@ __global__ void __launch_bounds__(kGramThreads, 2)
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     float4* rowp = reinterpret_cast<float4*>(wdst + (int64_t)(8 * ty + i) * 128 + 8 * tx);
-    rowp[0] = make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
-    rowp[1] = make_float4(a[i][4], a[i][5], a[i][6], a[i][7]);
+    // W feeds only the scans' tf32 contractions: stored rounded to tf32
+    rowp[0] = make_float4(round_tf32(a[i][0]), round_tf32(a[i][1]), round_tf32(a[i][2]),
+                          round_tf32(a[i][3]));
+    rowp[1] = make_float4(round_tf32(a[i][4]), round_tf32(a[i][5]), round_tf32(a[i][6]),
+                          round_tf32(a[i][7]));
   }
 }
 
@@ -391,21 +394,24 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     const uint32_t sW = base + kScanSmemW + (uint32_t)st * 65536u;
     const uint32_t sX = base + kScanSmemX + (uint32_t)st * 32768u;
     if (!mbar_wait(full[st], (uint32_t)((s >> 1) & 1))) { ok = false; break; }
-    if (s > 0) {
-      // X^T[n][i] = C^T[n][i] + lambda S_prev[i][n]
+    {
+      // X^T[n][i] = C^T[n][i] + lambda S_prev[i][n] (no state before the text
+      // step), rounded to tf32 here so the contraction does not truncate it
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(c * 32), sv);
-        tmem_ld_wait(sv);
+        if (s > 0) {
+          tmem_ld32(tmem + lane_base + (uint32_t)(c * 32), sv);
+          tmem_ld_wait(sv);
+        }
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
           const uint32_t n = (uint32_t)(c * 32 + jj);
           const uint32_t addr = sX + xcol + sw128_off(n, xu);
           float x;
           asm volatile("ld.shared.f32 %0, [%1];" : "=f"(x) : "r"(addr) : "memory");
-          x = fmaf(p.lambda, __uint_as_float(sv[jj]), x);
-          asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(x) : "memory");
+          if (s > 0) x = fmaf(p.lambda, __uint_as_float(sv[jj]), x);
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(round_tf32(x)) : "memory");
         }
       }
     }

@@ -361,6 +361,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// fp32 -> tf32 with round-to-nearest (ties away from zero), kept in an fp32
+// register (low 13 mantissa bits zero). tcgen05 kind::tf32 reads only the top
+// 19 bits of each operand, i.e. truncates; operands rounded here first carry
+// an unbiased error instead, which does not build up along a long scan.
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
