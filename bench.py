@@ -372,10 +372,16 @@ def run_profile(args) -> None:
         elif args.profile == "bsa":
             V.vdn_bsa_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"], o_soft, None,
                           ws)
+        elif args.profile == "merge":
+            V.vdn_gate_merge(shape, dev["q"], R, o_soft, dev["g_s"], dev["g_l"], rms_w, out, ws)
         else:
             V.vdn_vda_scan(shape, dev["k"], dev["v"], dev["kt"], dev["vt"], R, None, None, None,
                            ws)
 
+    if args.profile == "merge":
+        # the merge reads real read states and o_soft
+        V.vdn_vda_scan(shape, dev["k"], dev["v"], dev["kt"], dev["vt"], R, None, None, None, ws)
+        V.vdn_bsa_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"], o_soft, None, ws)
     for _ in range(args.warmup + args.steps):
         once()
     torch.cuda.synchronize()
@@ -435,7 +441,7 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--cpu-heads", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["layer", "bsa", "vda"],
+    ap.add_argument("--profile", choices=["layer", "bsa", "vda", "merge"],
                     help="only run launches of one entry point (for ncu captures)")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="workload name (vdn_synth.CONFIGS); the default is the headline one")
