@@ -404,13 +404,17 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           tmem_ld32(tmem + lane_base + (uint32_t)(c * 32), sv);
           tmem_ld_wait(sv);
         }
+        // all 32 loads first, so they overlap, then the updates and stores
+        float xv[32];
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
-          const uint32_t n = (uint32_t)(c * 32 + jj);
-          const uint32_t addr = sX + xcol + sw128_off(n, xu);
-          float x;
-          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(x) : "r"(addr) : "memory");
-          if (s > 0) x = fmaf(p.lambda, __uint_as_float(sv[jj]), x);
+          const uint32_t addr = sX + xcol + sw128_off((uint32_t)(c * 32 + jj), xu);
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(xv[jj]) : "r"(addr) : "memory");
+        }
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const uint32_t addr = sX + xcol + sw128_off((uint32_t)(c * 32 + jj), xu);
+          const float x = (s > 0) ? fmaf(p.lambda, __uint_as_float(sv[jj]), xv[jj]) : xv[jj];
           asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(round_tf32(x)) : "memory");
         }
       }
