@@ -227,11 +227,14 @@ def test_layer_deterministic():
     assert torch.equal(a, b)
 
 
-def test_gate_merge_entry_matches_layer():
-    # softmax branch + scan + gate merge called separately == whole layer
+@pytest.mark.parametrize("d", [128, 64])
+def test_gate_merge_entry_matches_layer(d):
+    # softmax branch + scan + gate merge called separately == whole layer and
+    # the oracle (d = 128 bf16 runs the TMA-streamed merge kernel, d = 64 the
+    # row-per-thread one)
     import video_diffusion_hybrid_block_b200 as V
     from vdn_cases import make_shape
-    inp = mid_case(seed=5)
+    inp = mid_case(seed=5, d=d)
     dev = device_inputs(inp)
     o, _ = run_bsa(inp, dev)
     R, _, _, _ = run_scan(inp, dev, per_frame=False)
@@ -243,3 +246,7 @@ def test_gate_merge_entry_matches_layer():
     got = out.float().cpu().numpy()
     ref = full.float().cpu().numpy()
     assert rel_l2(got, ref) <= 1e-2
+    for h in range(inp["H"]):
+        oref = O.layer_head(inp, h)["out"]
+        assert rel_l2(got[:, h], oref) <= OUT_REL_L2, h
+        assert max_abs(got[:, h], oref) <= OUT_MAX_ABS, h

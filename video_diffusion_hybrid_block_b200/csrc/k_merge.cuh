@@ -213,4 +213,224 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   }
 }
 
+// Same operation for the common case (bf16 out, d = 128, o_soft [N, H, 128]
+// bf16), streamed and warp-specialised. Warp 4 (one thread) runs a three-stage
+// TMA ring of (q, o_soft) tiles two tiles ahead of the contractions and issues
+// o_lin = q R_b into a double-buffered TMEM accumulator; warps 0-3 run the
+// epilogue (thread = row = TMEM lane) and never wait on a load. A full tile
+// of `out` is written into the q buffer of its stage (already consumed by the
+// contraction) and leaves through one TMA store; a block's ragged last tile
+// is stored row by row. Hand-offs: in_full/in_empty per stage, acc_full /
+// acc_empty per TMEM buffer.
+constexpr int kMergeTmaThreads = 160;
+constexpr int kMergeTmaStages = 3;
+constexpr int kMergeTmaTiles = 14;           // 3 CTAs cover a 40-tile block
+constexpr uint32_t kMergeTmaSmemR = 0;       // 32 KB
+constexpr uint32_t kMergeTmaSmemQ = 32768;   // stage s: Q at 32 KB + 64 KB s, O_soft 32 KB after it
+constexpr uint32_t kMergeTmaSmemBytes = (1 + 2 * kMergeTmaStages) * 32768 + 1024;
+
+__global__ void __launch_bounds__(kMergeTmaThreads, 1)
+    k_readout_merge_tma(const __grid_constant__ CUtensorMap tq,
+                        const __grid_constant__ CUtensorMap tos,
+                        const __grid_constant__ CUtensorMap tout, const MergeParams p) {
+  const int b = blockIdx.y, h = blockIdx.z;
+  int q0, q1;
+  block_rows(p.off, p.F, p.bf, b, q0, q1);
+  const int t_first = blockIdx.x * kMergeTmaTiles;
+  const int ntl = imin(kMergeTmaTiles, (q1 - q0 + kTile - 1) / kTile - t_first);
+  if (ntl <= 0) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t in_full[kMergeTmaStages], in_empty[kMergeTmaStages], acc_full[2], acc_empty[2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ float wsm[128];
+  __shared__ int abort_flag;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sR = base + kMergeTmaSmemR;
+  const int i = threadIdx.x, warp = i >> 5;
+  auto sQ = [&](int st) { return base + kMergeTmaSmemQ + (uint32_t)st * 65536u; };
+  auto sO = [&](int st) { return base + kMergeTmaSmemQ + (uint32_t)st * 65536u + 32768u; };
+
+  if (i == 0) {
+    abort_flag = 0;
+    for (int k = 0; k < kMergeTmaStages; ++k) {
+      mbar_init(smem_u32(&in_full[k]), 1);
+      mbar_init(smem_u32(&in_empty[k]), 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(smem_u32(&acc_full[k]), 1);
+      mbar_init(smem_u32(&acc_empty[k]), 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  volatile int* abort_v = &abort_flag;
+
+  if (warp == 4) {
+    // ------------------------------------------------ loads and contractions
+    if (i == 128) {
+      auto load_tile = [&](int t) {
+        const int st = t % kMergeTmaStages;
+        const uint32_t bar = smem_u32(&in_full[st]);
+        mbar_arrive_expect_tx(bar, 65536);
+        const int row = q0 + (t_first + t) * kTile;
+        tma_load_3d(sQ(st), &tq, bar, 0, h, row);
+        tma_load_3d(sQ(st) + 16384, &tq, bar, 64, h, row);
+        tma_load_3d(sO(st), &tos, bar, 0, h, row);
+        tma_load_3d(sO(st) + 16384, &tos, bar, 64, h, row);
+      };
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tos);
+      tma_prefetch_desc(&tout);
+      for (int t = 0; t < imin(ntl, kMergeTmaStages); ++t) load_tile(t);
+    }
+    // R_b is ready once the epilogue warps pass this barrier
+    named_barrier_sync(1, kMergeTmaThreads);
+    if (i == 128) {
+      const uint32_t idO = idesc_bf16(128, 128, false, true);
+      for (int t = 0; t < ntl; ++t) {
+        if (*abort_v) break;
+        const int st = t % kMergeTmaStages, ab = t & 1;
+        if (!mbar_wait(smem_u32(&in_full[st]), (uint32_t)((t / kMergeTmaStages) & 1))) {
+          *abort_v = 1;
+          break;
+        }
+        if (t >= 2 && !mbar_wait(smem_u32(&acc_empty[ab]), (uint32_t)(((t - 2) >> 1) & 1))) {
+          *abort_v = 1;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          umma_bf16_ss(tmem + (uint32_t)(ab * 128),
+                       sdesc_sw128(sQ(st) + (uint32_t)((s >> 2) * 16384 + (s & 3) * 32), 16, 1024),
+                       sdesc_sw128(sR + (uint32_t)(s * 2048), 16384, 1024), idO, s > 0 ? 1u : 0u);
+        umma_commit(smem_u32(&acc_full[ab]));
+        // refill the stage of tile t-1 once its epilogue is done with it
+        const int tn = t + kMergeTmaStages - 1;
+        if (t >= 1 && tn < ntl) {
+          const int sp = (t - 1) % kMergeTmaStages;
+          if (!mbar_wait(smem_u32(&in_empty[sp]), (uint32_t)(((t - 1) / kMergeTmaStages) & 1))) {
+            *abort_v = 1;
+            break;
+          }
+          const uint32_t bar = smem_u32(&in_full[sp]);
+          mbar_arrive_expect_tx(bar, 65536);
+          const int row = q0 + (t_first + tn) * kTile;
+          tma_load_3d(sQ(sp), &tq, bar, 0, h, row);
+          tma_load_3d(sQ(sp) + 16384, &tq, bar, 64, h, row);
+          tma_load_3d(sO(sp), &tos, bar, 0, h, row);
+          tma_load_3d(sO(sp) + 16384, &tos, bar, 64, h, row);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // R_b (fwd + bwd) -> bf16, row i (key dim), MN-major 128B-swizzled
+    const int64_t rbase = ((int64_t)b * p.H + h) * 128 * 128;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float4* ra = reinterpret_cast<const float4*>(p.RA + rbase + (int64_t)i * 128 + c * 64 + u * 8);
+        float4 x0 = __ldg(ra), x1 = __ldg(ra + 1);
+        if (p.RB) {
+          const float4* rb = reinterpret_cast<const float4*>(p.RB + rbase + (int64_t)i * 128 + c * 64 + u * 8);
+          const float4 y0 = __ldg(rb), y1 = __ldg(rb + 1);
+          x0 = make_float4(x0.x + y0.x, x0.y + y0.y, x0.z + y0.z, x0.w + y0.w);
+          x1 = make_float4(x1.x + y1.x, x1.y + y1.y, x1.z + y1.z, x1.w + y1.w);
+        }
+        st_shared_v4(sR + (uint32_t)(c * 16384) + sw128_off((uint32_t)i, (uint32_t)u),
+                     pack_bf16x2(x0.x, x0.y), pack_bf16x2(x0.z, x0.w), pack_bf16x2(x1.x, x1.y),
+                     pack_bf16x2(x1.z, x1.w));
+      }
+    }
+    wsm[i] = __ldg(p.rms_w + (int64_t)h * 128 + i);
+    fence_proxy_async_smem();
+    named_barrier_sync(1, kMergeTmaThreads);
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    for (int t = 0; t < ntl; ++t) {
+      if (*abort_v) break;
+      const int st = t % kMergeTmaStages, ab = t & 1;
+      const int row0 = q0 + (t_first + t) * kTile;
+      const int row = row0 + i;
+      const bool valid = row < q1;
+      const bool full_tile = row0 + kTile <= q1;
+      float gsv = 0.f, glv = 0.f;
+      if (valid) {
+        gsv = sigmoidf_(load_gate(p.g_s, (int64_t)row * p.H + h, p.gate_f32));
+        glv = sigmoidf_(load_gate(p.g_l, (int64_t)row * p.H + h, p.gate_f32));
+      }
+      if (!mbar_wait(smem_u32(&acc_full[ab]), (uint32_t)((t >> 1) & 1))) { *abort_v = 1; break; }
+      tc_fence_after();
+      const uint32_t tO = tmem + lane_base + (uint32_t)(ab * 128);
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + (uint32_t)(c * 32), o);
+        tmem_ld_wait(o);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(o[e]), __uint_as_float(o[e]), ss);
+      }
+      const float nr = glv * rsqrtf(ss * (1.f / 128.f) + p.eps);
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + ((int64_t)row * p.H + h) * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + (uint32_t)(c * 32), o);
+        tmem_ld_wait(o);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c0 = c * 32 + u * 8;
+          const uint32_t off = (uint32_t)(c0 >> 6) * 16384u + sw128_off((uint32_t)i, (uint32_t)((c0 & 63) >> 3));
+          const uint4 ov = ld_shared_v4(sO(st) + off);
+          const uint32_t w4[4] = {ov.x, ov.y, ov.z, ov.w};
+          uint32_t y4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int cc = c0 + 2 * e;
+            const float ylo = gsv * bf_lo(w4[e]) + nr * wsm[cc] * __uint_as_float(o[u * 8 + 2 * e]);
+            const float yhi = gsv * bf_hi(w4[e]) + nr * wsm[cc + 1] * __uint_as_float(o[u * 8 + 2 * e + 1]);
+            y4[e] = pack_bf16x2(ylo, yhi);
+          }
+          if (full_tile)
+            st_shared_v4(sQ(st) + off, y4[0], y4[1], y4[2], y4[3]);  // Q_t is consumed
+          else if (valid)
+            *reinterpret_cast<uint4*>(orow + c0) = make_uint4(y4[0], y4[1], y4[2], y4[3]);
+        }
+      }
+      // TMEM buffer ab is read: the contraction of tile t+2 may overwrite it
+      tc_fence_before();
+      fence_proxy_async_smem();
+      named_barrier_sync(2, 128);
+      if (i == 0) {
+        mbar_arrive(smem_u32(&acc_empty[ab]));
+        if (full_tile) {
+          tma_store_3d(&tout, sQ(st), 0, h, row0);
+          tma_store_3d(&tout, sQ(st) + 16384, 64, h, row0);
+          bulk_commit_group();
+          bulk_wait_read_all();  // the stage may be refilled once the store has read it
+        }
+        mbar_arrive(smem_u32(&in_empty[st]));
+      }
+    }
+    if (i == 0) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 }  // namespace vdn

@@ -159,6 +159,8 @@ bool set_smem_attrs() {
                                   (int)kScanSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_readout_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kMergeSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_readout_merge_tma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kMergeTmaSmemBytes) == cudaSuccess;
   done[dev] = ok;
   return ok;
 }
@@ -350,6 +352,18 @@ int launch_merge(const Plan& P, const __nv_bfloat16* qb, const float* RA, const 
   mp.eps = P.eps;
   mp.out = out;
   mp.out_f32 = (P.dtype == VDN_F32);
+  // bf16 out, d = 128, packed o_soft [N, H, 128]: streamed variant (TMA in and out)
+  if (P.dtype == VDN_BF16 && P.d == kDPad && r_d == kDPad && os_head == kDPad &&
+      os_row == (int64_t)P.H * kDPad) {
+    CUtensorMap tos, tout;
+    if (!act_map(&tos, o_soft, P.N, P, 128, ws + P.o_C) ||
+        !act_map(&tout, out, P.N, P, 128, ws + P.o_C))
+      return VDN_ERR_CUDA;
+    const int gx = (P.max_qtiles + kMergeTmaTiles - 1) / kMergeTmaTiles;
+    k_readout_merge_tma<<<dim3(gx, P.nb, P.H), kMergeTmaThreads, kMergeTmaSmemBytes, st>>>(tq, tos,
+                                                                                      tout, mp);
+    return VDN_OK;
+  }
   const int gx = (P.max_qtiles + kMergeTiles - 1) / kMergeTiles;
   k_readout_merge<<<dim3(gx, P.nb, P.H), kMergeThreads, kMergeSmemBytes, st>>>(tq, mp);
   return VDN_OK;
