@@ -17,9 +17,10 @@
 //   L2-normalises k rows in shared memory, accumulates G = K^T K and
 //   C^T = V^T K as two M=128 x N=128 bf16 tcgen05 contractions into TMEM,
 //   writes C^T (fp32, the layout the scan loads as its X operand)
-//   and then inverts M = lambda I + G in registers with a Gauss-Jordan sweep
-//   (no pivoting: M is symmetric positive definite with eigenvalues
-//   >= lambda) and writes W = M^-1 (fp32).
+//   and then inverts M = lambda I + G (2 x 2 blocks of 64: two 64-pivot
+//   Gauss-Jordan sweeps in registers, no pivoting since M is symmetric
+//   positive definite with eigenvalues >= lambda, and four 64^3 products
+//   through the Schur complement) and writes W = M^-1 (fp32, tf32-rounded).
 // Only frames whose state some block reads are processed: the forward scan
 //   stops at the largest forward read index, the backward scan at the
 //   smallest backward one (the remaining frames always sit inside the window
@@ -230,80 +231,168 @@ __global__ void __launch_bounds__(kGramThreads, 2)
     tmem_dealloc(tmem, 256);
   }
 
-  // Gauss-Jordan inverse of M = lambda I + G: thread (ty, tx) holds the 8 x 8
-  // tile rows 8ty.., columns 8tx.. (16 x 16 threads), one barrier per pivot.
+  // Inverse of M = lambda I + G = [[A, B], [B^T, D]] (64 x 64 blocks) by the
+  // Schur complement: X = A^-1 B, S = D - B^T X, Y = X S^-1, and
+  //   W = M^-1 = [[A^-1 + Y X^T, -Y], [-Y^T, S^-1]].
+  // A^-1 and S^-1 come from 64-pivot Gauss-Jordan sweeps (no pivoting: both
+  // are symmetric positive definite with eigenvalues >= lambda) on 4 x 4
+  // register tiles, thread (ty, tx) holding rows 4ty.., columns 4tx..; the
+  // four 64 x 64 x 64 products are sums of rank-1 updates read from shared
+  // memory as 16-byte vectors (A^-1 is symmetric; X and Y are also kept
+  // transposed). W feeds only the scans' tf32 contractions and is stored
+  // rounded to tf32.
   const int ty = tid >> 4, tx = tid & 15;
-  float a[8][8];
+  // G element (r, c) in the swizzled copy: row r at 512 r, 16-byte unit c / 4
+  auto g_addr = [&](int r, int c) -> uint32_t {
+    return gs + (uint32_t)r * 512u + ((((uint32_t)(c >> 2)) ^ ((uint32_t)r & 31u)) << 4);
+  };
+  // 64 x 64 fp32 matrices, row-major (256 B rows): AI and X beyond G (bytes
+  // 64K..96K of the staging area); SI, XT and YT over G once it is consumed
+  const uint32_t mAI = base + 65536u, mX = base + 81920u;
+  const uint32_t mSI = base, mXT = base + 16384u, mYT = base + 32768u;
+  auto m_addr = [](uint32_t m, int r, int c) -> uint32_t { return m + (uint32_t)(r * 64 + c) * 4u; };
+  auto ld4 = [](uint32_t addr) -> float4 {
+    const uint4 v = ld_shared_v4(addr);
+    return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+  };
+  auto st4 = [](uint32_t addr, float x0, float x1, float x2, float x3) {
+    st_shared_v4(addr, __float_as_uint(x0), __float_as_uint(x1), __float_as_uint(x2), __float_as_uint(x3));
+  };
+  // in-place Gauss-Jordan inverse of a 64 x 64 SPD matrix held in 4 x 4 tiles
+  auto gj64 = [&](float (&a)[4][4]) {
+    for (int kb = 0; kb < 16; ++kb) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t R = (uint32_t)(8 * ty + i);
+      for (int kk = 0; kk < 4; ++kk) {
+        const int k = kb * 4 + kk;
+        const int buf = k & 1;
+        if (ty == kb)
+          *reinterpret_cast<float4*>(&rowbuf[buf][4 * tx]) = make_float4(a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
+        if (tx == kb)
+          *reinterpret_cast<float4*>(&colbuf[buf][4 * ty]) = make_float4(a[0][kk], a[1][kk], a[2][kk], a[3][kk]);
+        __syncthreads();
+        const float ip = 1.f / rowbuf[buf][k];
+        const float4 r4 = *reinterpret_cast<const float4*>(&rowbuf[buf][4 * tx]);
+        const float4 c4 = *reinterpret_cast<const float4*>(&colbuf[buf][4 * ty]);
+        const float rj[4] = {r4.x * ip, r4.y * ip, r4.z * ip, r4.w * ip};
+        const float ci[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-    for (int hlf = 0; hlf < 2; ++hlf) {
-      const uint4 v = ld_shared_v4(gs + R * 512u + ((((uint32_t)(2 * tx + hlf)) ^ (R & 31u)) << 4));
-      a[i][4 * hlf + 0] = __uint_as_float(v.x);
-      a[i][4 * hlf + 1] = __uint_as_float(v.y);
-      a[i][4 * hlf + 2] = __uint_as_float(v.z);
-      a[i][4 * hlf + 3] = __uint_as_float(v.w);
+        for (int i = 0; i < 4; ++i) {
+          const float2 nc = make_float2(-ci[i], -ci[i]);
+#pragma unroll
+          for (int j = 0; j < 4; j += 2) {
+            const float2 upd = ffma2(nc, make_float2(rj[j], rj[j + 1]), make_float2(a[i][j], a[i][j + 1]));
+            a[i][j] = upd.x;
+            a[i][j + 1] = upd.y;
+          }
+        }
+        if (ty == kb) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) a[kk][j] = rj[j];
+        }
+        if (tx == kb) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a[i][kk] = -ci[i] * ip;
+        }
+        if (ty == kb && tx == kb) a[kk][kk] = ip;
+      }
     }
+  };
+  // acc[i][j] += sum_k P[4ty+i][k] Q[k][4tx+j], with colP(k) = P[4ty..4ty+3][k]
+  // and rowQ(k) = Q[k][4tx..4tx+3] as 16-byte vectors
+  auto mm_acc = [&](float (&acc)[4][4], auto colP, auto rowQ) {
+#pragma unroll 8
+    for (int k = 0; k < 64; ++k) {
+      const float4 pv = colP(k);
+      const float4 q = rowQ(k);
+      const float pi[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 pp = make_float2(pi[i], pi[i]);
+        const float2 u0 = ffma2(pp, make_float2(q.x, q.y), make_float2(acc[i][0], acc[i][1]));
+        const float2 u1 = ffma2(pp, make_float2(q.z, q.w), make_float2(acc[i][2], acc[i][3]));
+        acc[i][0] = u0.x;
+        acc[i][1] = u0.y;
+        acc[i][2] = u1.x;
+        acc[i][3] = u1.y;
+      }
+    }
+  };
+  float* wdst = p.Wmat + ((int64_t)m * p.H + h) * 128 * 128;
+  auto store_w = [&](int r, int c0, float x0, float x1, float x2, float x3) {
+    *reinterpret_cast<float4*>(wdst + (int64_t)r * 128 + c0) =
+        make_float4(round_tf32(x0), round_tf32(x1), round_tf32(x2), round_tf32(x3));
+  };
+
+  // 1. A^-1 (kept in registers for step 7 too)
+  float ai[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 v = ld4(g_addr(4 * ty + i, 4 * tx));
+    ai[i][0] = v.x; ai[i][1] = v.y; ai[i][2] = v.z; ai[i][3] = v.w;
   }
   if (ty == tx) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a[i][i] += p.lambda;
+    for (int i = 0; i < 4; ++i) ai[i][i] += p.lambda;
   }
-  for (int kb8 = 0; kb8 < 16; ++kb8) {
+  gj64(ai);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const int k = kb8 * 8 + kk;
-      const int buf = k & 1;
-      if (ty == kb8) {
-        *reinterpret_cast<float4*>(&rowbuf[buf][8 * tx]) = make_float4(a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
-        *reinterpret_cast<float4*>(&rowbuf[buf][8 * tx + 4]) = make_float4(a[kk][4], a[kk][5], a[kk][6], a[kk][7]);
-      }
-      if (tx == kb8) {
-        *reinterpret_cast<float4*>(&colbuf[buf][8 * ty]) = make_float4(a[0][kk], a[1][kk], a[2][kk], a[3][kk]);
-        *reinterpret_cast<float4*>(&colbuf[buf][8 * ty + 4]) = make_float4(a[4][kk], a[5][kk], a[6][kk], a[7][kk]);
-      }
-      __syncthreads();
-      const float ip = 1.f / rowbuf[buf][k];
-      const float4 r0 = *reinterpret_cast<const float4*>(&rowbuf[buf][8 * tx]);
-      const float4 r1 = *reinterpret_cast<const float4*>(&rowbuf[buf][8 * tx + 4]);
-      const float4 c0 = *reinterpret_cast<const float4*>(&colbuf[buf][8 * ty]);
-      const float4 c1 = *reinterpret_cast<const float4*>(&colbuf[buf][8 * ty + 4]);
-      const float rj[8] = {r0.x * ip, r0.y * ip, r0.z * ip, r0.w * ip,
-                           r1.x * ip, r1.y * ip, r1.z * ip, r1.w * ip};
-      const float ci[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      // rank-1 update a -= c r^T / pivot, two columns per instruction
+  for (int i = 0; i < 4; ++i) st4(m_addr(mAI, 4 * ty + i, 4 * tx), ai[i][0], ai[i][1], ai[i][2], ai[i][3]);
+  __syncthreads();
+  // 2. X = A^-1 B, B = G[0:64, 64:128]; column k of A^-1's row block = row k (symmetric)
+  float xt[4][4] = {};
+  mm_acc(xt, [&](int k) { return ld4(m_addr(mAI, k, 4 * ty)); },
+         [&](int k) { return ld4(g_addr(k, 64 + 4 * tx)); });
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float2 nc = make_float2(-ci[i], -ci[i]);
+  for (int i = 0; i < 4; ++i) st4(m_addr(mX, 4 * ty + i, 4 * tx), xt[i][0], xt[i][1], xt[i][2], xt[i][3]);
+  __syncthreads();
+  // 3. S = lambda I + G[64:128, 64:128] - B^T X; column k of B^T's row block = row k of B
+  float sa[4][4];
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-          const float2 upd = ffma2(nc, make_float2(rj[j], rj[j + 1]), make_float2(a[i][j], a[i][j + 1]));
-          a[i][j] = upd.x;
-          a[i][j + 1] = upd.y;
-        }
-      }
-      if (ty == kb8) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) a[kk][j] = rj[j];
-      }
-      if (tx == kb8) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a[i][kk] = -ci[i] * ip;
-      }
-      if (ty == kb8 && tx == kb8) a[kk][kk] = ip;
-    }
+  for (int i = 0; i < 4; ++i) {
+    const float4 v = ld4(g_addr(64 + 4 * ty + i, 64 + 4 * tx));
+    sa[i][0] = -v.x; sa[i][1] = -v.y; sa[i][2] = -v.z; sa[i][3] = -v.w;
   }
-  float* wdst = p.Wmat + ((int64_t)m * p.H + h) * 128 * 128;
+  if (ty == tx) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float4* rowp = reinterpret_cast<float4*>(wdst + (int64_t)(8 * ty + i) * 128 + 8 * tx);
-    // W feeds only the scans' tf32 contractions: stored rounded to tf32
-    rowp[0] = make_float4(round_tf32(a[i][0]), round_tf32(a[i][1]), round_tf32(a[i][2]),
-                          round_tf32(a[i][3]));
-    rowp[1] = make_float4(round_tf32(a[i][4]), round_tf32(a[i][5]), round_tf32(a[i][6]),
-                          round_tf32(a[i][7]));
+    for (int i = 0; i < 4; ++i) sa[i][i] -= p.lambda;
   }
+  mm_acc(sa, [&](int k) { return ld4(g_addr(k, 64 + 4 * ty)); },
+         [&](int k) { return ld4(m_addr(mX, k, 4 * tx)); });
+  // sa = B^T X - D; S = -sa
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sa[i][j] = -sa[i][j];
+  __syncthreads();  // G is consumed: SI, XT, YT may overwrite it
+  // X^T tile (this thread's X tile, transposed)
+#pragma unroll
+  for (int j = 0; j < 4; ++j) st4(m_addr(mXT, 4 * tx + j, 4 * ty), xt[0][j], xt[1][j], xt[2][j], xt[3][j]);
+  // 4. S^-1 = W[64:128, 64:128]
+  gj64(sa);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    st4(m_addr(mSI, 4 * ty + i, 4 * tx), sa[i][0], sa[i][1], sa[i][2], sa[i][3]);
+    store_w(64 + 4 * ty + i, 64 + 4 * tx, sa[i][0], sa[i][1], sa[i][2], sa[i][3]);
+  }
+  __syncthreads();
+  // 5. Y = X S^-1; W[0:64, 64:128] = -Y, W[64:128, 0:64] = -Y^T
+  float y[4][4] = {};
+  mm_acc(y, [&](int k) { return ld4(m_addr(mXT, k, 4 * ty)); },
+         [&](int k) { return ld4(m_addr(mSI, k, 4 * tx)); });
+#pragma unroll
+  for (int i = 0; i < 4; ++i) store_w(4 * ty + i, 64 + 4 * tx, -y[i][0], -y[i][1], -y[i][2], -y[i][3]);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    store_w(64 + 4 * tx + j, 4 * ty, -y[0][j], -y[1][j], -y[2][j], -y[3][j]);
+    st4(m_addr(mYT, 4 * tx + j, 4 * ty), y[0][j], y[1][j], y[2][j], y[3][j]);
+  }
+  __syncthreads();
+  // 6. W[0:64, 0:64] = A^-1 + Y X^T; column k of Y's row block = row k of Y^T,
+  //    row k of X^T = X^T[k][..]
+  mm_acc(ai, [&](int k) { return ld4(m_addr(mYT, k, 4 * ty)); },
+         [&](int k) { return ld4(m_addr(mXT, k, 4 * tx)); });
+#pragma unroll
+  for (int i = 0; i < 4; ++i) store_w(4 * ty + i, 4 * tx, ai[i][0], ai[i][1], ai[i][2], ai[i][3]);
 }
 
 // --------------------------------------------------------------- scans ----
