@@ -270,7 +270,10 @@ __global__ void __launch_bounds__(kGramThreads, 2)
         if (tx == kb)
           *reinterpret_cast<float4*>(&colbuf[buf][4 * ty]) = make_float4(a[0][kk], a[1][kk], a[2][kk], a[3][kk]);
         __syncthreads();
-        const float ip = 1.f / rowbuf[buf][k];
+        // pivot >= lambda > 0: the MUFU reciprocal (within a couple of ulp) is
+        // enough, and it shortens the per-pivot chain
+        float ip;
+        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(ip) : "f"(rowbuf[buf][k]));
         const float4 r4 = *reinterpret_cast<const float4*>(&rowbuf[buf][4 * tx]);
         const float4 c4 = *reinterpret_cast<const float4*>(&colbuf[buf][4 * ty]);
         const float rj[4] = {r4.x * ip, r4.y * ip, r4.z * ip, r4.w * ip};
