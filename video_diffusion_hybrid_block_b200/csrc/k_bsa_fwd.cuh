@@ -232,7 +232,6 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         umma_commit(smem_u32(&bar_ke[0]));
       }
       for (int j = 0; ok && j < nkt; ++j) {
-        if (*abort_v) { ok = false; break; }
         const int st = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         const int st1 = (j + 1) & 1;
@@ -288,7 +287,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
                       make_float2(0.f, 0.f)};
     bool ok = true;
     for (int j = 0; j < nkt; ++j) {
-      if (*abort_v) { ok = false; break; }
+      // no per-tile abort poll: a failed (bounded) wait ends the loop
       int src, row0, valid;
       segs_tile(segs, j, src, row0, valid);
       if (!mbar_wait(s_full, (uint32_t)(j & 1))) { ok = false; break; }
