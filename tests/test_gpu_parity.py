@@ -53,15 +53,29 @@ def _max_frames_case():
     return S.make_inputs_from(4096, sizes, 4, 1, 32, "bf16", seed=9)
 
 
+def _block_size_case(name):
+    """Blocks of one frame (the window is three frames) on ragged frames, and
+    blocks of seven frames."""
+    if name == "bf1":
+        inp = S.make_inputs_from(9, [37, 0, 5, 129, 64, 2, 90, 11, 40], 7, 2, 128, "bf16", seed=12)
+        inp["block_frames"] = 1
+    else:
+        inp = S.make_inputs_from(30, [110] * 30, 33, 2, 128, "bf16", seed=13)
+        inp["block_frames"] = 7
+    return inp
+
+
 def _edge(name):
     if name == "max-jump":
         return _max_jump_case()
     if name == "F4096":
         return _max_frames_case()
+    if name in ("bf1", "bf7"):
+        return _block_size_case(name)
     return dict(_edge_cases())[name]
 
 
-EDGE = [n for n, _ in _edge_cases()] + ["max-jump", "F4096"]
+EDGE = [n for n, _ in _edge_cases()] + ["max-jump", "F4096", "bf1", "bf7"]
 
 
 def _cases(name):

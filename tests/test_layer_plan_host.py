@@ -91,6 +91,9 @@ def _layouts():
         ("bf3", S.frame_offsets([130] * 14), 3, 40),
         ("F4096", S.frame_offsets(rng.integers(0, 4, size=4096)), 5, 4),
         ("big-frames", S.frame_offsets([1792] * 20), 5, 512),
+        ("bf1", S.frame_offsets([37, 0, 5, 129, 64, 2, 90, 11, 40]), 1, 7),
+        ("bf7", S.frame_offsets([110] * 30), 7, 33),
+        ("bf-larger-than-F", S.frame_offsets([20, 30, 0, 9]), 6, 3),
     ]
 
 
