@@ -63,9 +63,15 @@ def test_workspace_bytes(lib):
         off = S.frame_offsets(S.frame_sizes(cfg))
         n = V.vdn_workspace_bytes(shape(off, cfg["T"], cfg["H"], cfg["d"],
                                         dtype=0 if cfg["dtype"] == "bf16" else 1))
-        N = int(off[-1])
-        assert n >= N * cfg["H"] * 128 * 2  # at least the o_soft buffer
-        assert n % 256 == 0
+        N, F, H, T = int(off[-1]), len(off) - 1, cfg["H"], cfg["T"]
+        a256 = lambda x: -(-x // 256) * 256  # noqa: E731
+        staged = cfg["dtype"] != "bf16" or cfg["d"] != 128
+        nb = -(-F // 5)
+        want = (3 * a256(N * H * 256) + 2 * a256(T * H * 256) if staged else 0) \
+            + 2 * a256((F - 1) * H * 65536) + a256(2 * nb * H * 65536) + a256(nb * H * 32768)
+        # staged bf16 q,k,v,kt,vt (fp32 or d < 128 only), C and W per matrix,
+        # the two read-state halves, the packed read-state tiles
+        assert n == want, (name, n, want)
     assert V.vdn_workspace_bytes(shape(d=48)) == 0
     assert V.vdn_workspace_bytes(shape(off=[0, 5])) == 0   # F = 1
 

@@ -84,7 +84,7 @@ struct Plan {
   int dtype;
   int max_qtiles;
   bool staged;  // inputs are narrowed / padded into the workspace
-  size_t o_q, o_k, o_v, o_kt, o_vt, o_osoft, o_C, o_W, o_R, o_Rimg, total;
+  size_t o_q, o_k, o_v, o_kt, o_vt, o_C, o_W, o_R, o_Rimg, total;
   const int32_t* off_dev;
 };
 
@@ -132,7 +132,6 @@ int make_plan(const vdn_shape_t* s, Plan* P) {
   P->o_v = o; o += P->staged ? align256(act) : 0;
   P->o_kt = o; o += P->staged ? align256(txt) : 0;
   P->o_vt = o; o += P->staged ? align256(txt) : 0;
-  P->o_osoft = o; o += align256(act);
   P->o_C = o; o += align256(mat);
   P->o_W = o; o += align256(mat);
   P->o_R = o; o += align256((size_t)2 * P->nb * P->H * 128 * 128 * 4);
@@ -617,7 +616,7 @@ extern "C" int vdn_vda_scan_noalloc(const vdn_shape_t* shape, const void* k, con
   S.o_v = S.o_k + act;
   S.o_kt = S.o_v + act;
   S.o_vt = S.o_kt + txt;
-  S.o_q = S.o_osoft = 0;  // not used by the scan
+  S.o_q = 0;  // not used by the scan
   S.total = S.o_vt + txt;
   if (S.total > kNoAllocScratchBytes) return VDN_ERR_WORKSPACE_TOO_SMALL;
   uint8_t* scratch = nullptr;
