@@ -52,6 +52,22 @@ def layer_flops(inp: dict, soft_pairs: np.ndarray) -> dict:
                 total=softmax + grams + readout + solves)
 
 
+def vda_merge_roofline(inp: dict, layer_ms: float, softmax_ms: float, hbm_gbs: float) -> dict:
+    """VDA + merge path against its HBM roofline. Algorithmic bytes: k, v, kt,
+    vt read once, q, o_soft, g_s, g_l read and out written once (bf16). The
+    merge runs fused in the softmax kernel's epilogue, so the path's cost is
+    the layer time minus the softmax-only kernel."""
+    N, T, H, d = inp["N"], inp["T"], inp["H"], inp["d"]
+    act = N * H * d * 2
+    nbytes = 2 * act + 2 * T * H * d * 2 + 2 * act + 2 * N * H * 2 + act
+    roof_ms = nbytes / (hbm_gbs * 1e9) * 1e3
+    marginal = layer_ms - softmax_ms
+    return {"algorithmic_bytes": int(nbytes), "roofline_ms": round(roof_ms, 4),
+            "marginal_ms": round(marginal, 4),
+            "frac": round(roof_ms / marginal, 4) if marginal > 0 else None,
+            "method": "layer time minus the softmax-only kernel (merge fused in its epilogue)"}
+
+
 def workload_desc(name: str) -> str:
     if name == WORKLOAD:
         return WORKLOAD_DESC
@@ -337,6 +353,7 @@ def run_cuda(args) -> None:
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
+        "vda_merge": vda_merge_roofline(inp, ms, bsa_ms, peaks["hbm_gbs"]),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
         line["cpu_baseline"] = cpu_baseline(inp, fl, args.cpu_heads)

@@ -53,3 +53,12 @@ def test_workload_descriptions_and_l2_notes():
         assert name.split("-")[0] in bench.workload_desc(name)
     assert "> 126 MB L2" in bench.l2_note(400 * 2 ** 20)
     assert "fit in the 126 MB L2" in bench.l2_note(2 ** 20)
+
+
+def test_vda_merge_roofline_bytes():
+    # 625.7 MB at pages-scale: k, v, q, o_soft, out 124 MB each, kt, vt, gates
+    inp = S.make_inputs("pages-scale")
+    r = bench.vda_merge_roofline(inp, 2.766, 2.640, 6543.0)
+    assert r["algorithmic_bytes"] == 5 * 15120 * 32 * 128 * 2 + 2 * 256 * 32 * 128 * 2 + 2 * 15120 * 32 * 2
+    assert abs(r["roofline_ms"] - r["algorithmic_bytes"] / 6543e9 * 1e3) < 1e-4
+    assert abs(r["marginal_ms"] - 0.126) < 1e-9 and abs(r["frac"] - r["roofline_ms"] / 0.126) < 1e-3
