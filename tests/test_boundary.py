@@ -156,3 +156,34 @@ def test_binding_raises_on_error(lib):
 def test_selftest_wait_timeout_rejects_bad_arguments(lib, limit_ns, cols):
     # out-of-range limits or TMEM column counts fail before any launch
     assert lib.vdn_selftest_wait_timeout(limit_ns, cols, None) == -1
+
+
+def test_binding_rejects_tensors_the_kernels_would_overrun():
+    # The binding checks sizes, element sizes and device before calling the
+    # library: each case passes one host tensor (every other argument is a
+    # never-dereferenced address), so it raises before reaching the library.
+    import torch
+    off = S.frame_offsets([24] * 10)
+    sh = shape(off, T=8, H=2, d=128)            # bf16
+    N = int(off[-1])
+    act = N * 2 * 128
+    t = lambda n, dt=torch.bfloat16: torch.zeros(n, dtype=dt)  # noqa: E731
+    names = ("q", "k", "v", "kt", "vt", "g_s", "g_l", "rms_w", "out")
+
+    def call(**kw):
+        a = {n: FAKE for n in names}
+        a.update(kw)
+        V.vdn_hybrid_attn_fwd(sh, *(a[n] for n in names), FAKE, ws_bytes=1 << 40)
+    with pytest.raises(ValueError, match="q: .* elements"):
+        call(q=t(act - 1))
+    with pytest.raises(ValueError, match="k: elements of 4 bytes, expected 2"):
+        call(k=t(act, torch.float32))
+    with pytest.raises(ValueError, match="rms_w: .* elements"):
+        call(rms_w=t(2 * 128 - 8, torch.float32))
+    with pytest.raises(ValueError, match="out: must be a CUDA tensor"):
+        call(out=t(act))
+    with pytest.raises(ValueError, match="read_states"):
+        V.vdn_vda_scan(sh, FAKE, FAKE, FAKE, FAKE, t(1, torch.float32), None, None, None, FAKE,
+                       ws_bytes=1 << 40)
+    with pytest.raises(ValueError, match="soft_pairs"):
+        V.vdn_pair_audit(sh, t(10 * 10, torch.int64), FAKE)

@@ -99,6 +99,39 @@ def _ptr(t) -> int:
     return t.data_ptr()
 
 
+def _need(t, count: int, esize: int, name: str):
+    """Reject a tensor the kernels would read or write beyond its end: fewer
+    elements than the shape needs, a different element size, or host memory.
+    Larger tensors are accepted; ints (raw addresses) and None pass through."""
+    if t is None or isinstance(t, int):
+        return
+    if t.numel() < count:
+        raise ValueError(f"{name}: {t.numel()} elements, the shape needs {count}")
+    if t.element_size() != esize:
+        raise ValueError(f"{name}: elements of {t.element_size()} bytes, expected {esize}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+
+
+def _check_acts(shape, q=None, k=None, v=None, kt=None, vt=None, g_s=None, g_l=None, out=None):
+    e = 2 if shape.dtype == VDN_BF16 else 4
+    act, txt, gate = shape.N * shape.H * shape.d, shape.T * shape.H * shape.d, shape.N * shape.H
+    for t, n, name in ((q, act, "q"), (k, act, "k"), (v, act, "v"), (out, act, "out"),
+                       (g_s, gate, "g_s"), (g_l, gate, "g_l")):
+        _need(t, n, e, name)
+    if shape.T > 0:
+        _need(kt, txt, e, "kt")
+        _need(vt, txt, e, "vt")
+
+
+def _check_states(shape, read_states=None, text_state=None, fwd_states=None, bwd_states=None):
+    dd = shape.H * shape.d * shape.d
+    _need(read_states, shape.nb * dd, 4, "read_states")
+    _need(text_state, dd, 4, "text_state")
+    _need(fwd_states, shape.F * dd, 4, "fwd_states")
+    _need(bwd_states, shape.F * dd, 4, "bwd_states")
+
+
 def _nbytes(workspace, ws_bytes) -> int:
     if ws_bytes is not None:
         return int(ws_bytes)
@@ -127,6 +160,7 @@ class Shape:
         self.F = len(self.off_host) - 1
         self.N = int(self.off_host[-1])
         self.T, self.H, self.d = int(T), int(H), int(d)
+        self.dtype = int(dtype)
         self.block_frames = int(block_frames)
         self.nb = -(-self.F // self.block_frames) if self.block_frames > 0 else 0
         self.c = vdn_shape_t(
@@ -151,6 +185,8 @@ def vdn_workspace_bytes(shape: Shape) -> int:
 
 def vdn_hybrid_attn_fwd(shape: Shape, q, k, v, kt, vt, g_s, g_l, rms_w, out, workspace,
                         stream=None, ws_bytes=None):
+    _check_acts(shape, q, k, v, kt, vt, g_s, g_l, out)
+    _need(rms_w, shape.H * shape.d, 4, "rms_w")
     rc = load_library().vdn_hybrid_attn_fwd(
         shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(g_s), _ptr(g_l),
         _ptr(rms_w), _ptr(out), _ptr(workspace), _nbytes(workspace, ws_bytes),
@@ -161,6 +197,8 @@ def vdn_hybrid_attn_fwd(shape: Shape, q, k, v, kt, vt, g_s, g_l, rms_w, out, wor
 
 def vdn_vda_scan(shape: Shape, k, v, kt, vt, read_states, text_state, fwd_states, bwd_states,
                  workspace, stream=None, ws_bytes=None):
+    _check_acts(shape, k=k, v=v, kt=kt, vt=vt)
+    _check_states(shape, read_states, text_state, fwd_states, bwd_states)
     rc = load_library().vdn_vda_scan(
         shape.ref, _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(read_states), _ptr(text_state),
         _ptr(fwd_states), _ptr(bwd_states), _ptr(workspace),
@@ -173,6 +211,8 @@ def vdn_vda_scan_noalloc(shape: Shape, k, v, kt, vt, read_states, text_state, fw
                          bwd_states, stream=None):
     """vdn_vda_scan without a workspace argument: the library's built-in
     64 MiB device scratch is used instead (see include/vdn.h for the limit)."""
+    _check_acts(shape, k=k, v=v, kt=kt, vt=vt)
+    _check_states(shape, read_states, text_state, fwd_states, bwd_states)
     rc = load_library().vdn_vda_scan_noalloc(
         shape.ref, _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(read_states), _ptr(text_state),
         _ptr(fwd_states), _ptr(bwd_states), _stream(stream))
@@ -182,6 +222,10 @@ def vdn_vda_scan_noalloc(shape: Shape, k, v, kt, vt, read_states, text_state, fw
 
 def vdn_gate_merge(shape: Shape, q, read_states, o_soft, g_s, g_l, rms_w, out, workspace,
                    stream=None, ws_bytes=None):
+    _check_acts(shape, q=q, g_s=g_s, g_l=g_l, out=out)
+    _check_states(shape, read_states)
+    _need(o_soft, shape.N * shape.H * shape.d, 2, "o_soft")
+    _need(rms_w, shape.H * shape.d, 4, "rms_w")
     rc = load_library().vdn_gate_merge(
         shape.ref, _ptr(q), _ptr(read_states), _ptr(o_soft), _ptr(g_s), _ptr(g_l), _ptr(rms_w),
         _ptr(out), _ptr(workspace), _nbytes(workspace, ws_bytes),
@@ -192,6 +236,9 @@ def vdn_gate_merge(shape: Shape, q, read_states, o_soft, g_s, g_l, rms_w, out, w
 
 def vdn_bsa_fwd(shape: Shape, q, k, v, kt, vt, o_soft, lse, workspace, stream=None,
                 ws_bytes=None):
+    _check_acts(shape, q, k, v, kt, vt)
+    _need(o_soft, shape.N * shape.H * shape.d, 2, "o_soft")
+    _need(lse, shape.H * shape.N, 4, "lse")
     rc = load_library().vdn_bsa_fwd(
         shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(o_soft), _ptr(lse),
         _ptr(workspace), _nbytes(workspace, ws_bytes), _stream(stream))
@@ -200,6 +247,8 @@ def vdn_bsa_fwd(shape: Shape, q, k, v, kt, vt, o_soft, lse, workspace, stream=No
 
 
 def vdn_pair_audit(shape: Shape, soft_pairs, lin_pairs, stream=None):
+    _need(soft_pairs, shape.F * (shape.F + 1), 8, "soft_pairs")
+    _need(lin_pairs, shape.F * shape.F, 8, "lin_pairs")
     rc = load_library().vdn_pair_audit(shape.ref, _ptr(soft_pairs), _ptr(lin_pairs),
                                        _stream(stream))
     _check(rc, "vdn_pair_audit")
