@@ -13,7 +13,7 @@
 //
 // k_vda_gram_inv: one CTA per (matrix m, head): m = 0 is the text, m = f is
 //   latent frame f (1 <= f <= F-2; anchors 0 and F-1 are never scanned).
-//   Streams the frame's k, v rows in 64-token tiles (TMA, 2 stages),
+//   Streams the frame's k, v rows in 64-token tiles (TMA, 3-stage ring),
 //   L2-normalises k rows in shared memory, accumulates G = K^T K and
 //   C^T = V^T K as two M=128 x N=128 bf16 tcgen05 contractions into TMEM,
 //   writes C^T (fp32, the layout the scan loads as its X operand)
