@@ -142,17 +142,23 @@ int vdn_pair_audit(const vdn_shape_t* shape, int64_t* soft_pairs,
                    int64_t* lin_pairs, void* stream);
 
 /* Same results as vdn_vda_scan, for callers that cannot provide a workspace
- * (no paper counterpart: this is a deployment variant). Its scratch is a
+ * (no paper counterpart: this is a deployment variant). Such callers are,
+ * for instance, serving loops that cannot absorb the device-wide
+ * synchronisation cudaMalloc / cudaFree imply, or plug-ins whose process
+ * memory belongs to an allocator they have no handle to. Its scratch is a
  * 64 MiB array inside the library, resident on every GPU that loads the
  * library until the process exits; the call itself allocates nothing.
  * Limit: 128 KiB x H x (F - 1) for the per-frame matrices, plus
  * 128 KiB x H x ceil(F / block_frames) for the read states, plus (fp32 or
  * d < 128 inputs only) 256 B x H x (2N + 2T) of staged keys/values must fit
  * in 64 MiB; larger shapes return VDN_ERR_WORKSPACE_TOO_SMALL. The first call
- * on a device looks up the array's device address (cudaGetSymbolAddress), so
- * make that first call before any stream capture. All calls share the one
- * array: calls that overlap on the GPU (other streams, other host threads)
- * race and must be ordered by the caller. */
+ * in a CUDA context (normally once per device) looks up the array's device
+ * address with cudaGetSymbolAddress, so make that first call before any
+ * stream capture. All calls share the one array and every call overwrites
+ * what it reads: calls that overlap on the GPU (other streams, other host
+ * threads) race and must be ordered by the caller. Like every entry point
+ * here it makes CUDA runtime calls, so it may not be called from a stream
+ * host function (cudaLaunchHostFunc). */
 int vdn_vda_scan_noalloc(const vdn_shape_t* shape, const void* k, const void* v,
                          const void* kt, const void* vt, float* read_states,
                          float* text_state, float* fwd_states, float* bwd_states,

@@ -339,3 +339,75 @@ def test_linear_branch_normalises_keys():
     np.testing.assert_allclose(a["R"], b["R"], rtol=0, atol=1e-12)
     for f in a["fwd"]:
         np.testing.assert_allclose(a["fwd"][f], b["fwd"][f], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------- readout orientation, text start --
+
+def test_readout_is_q_transpose_state_one_token_closed_form():
+    # One video token (unit key k, value v) in frame 5 and no text: the
+    # forward state after it is (I + k k^T)^-1 k v^T = k v^T / 2 (lambda = 1,
+    # Sherman-Morrison), and frames 1..9 are the whole forward range block 3
+    # of a 20-frame clip reads (its window is frames 10..19; its backward
+    # read is the text state, here zero). A query q = k in block 3 must read
+    # o_lin = q^T R = (k.k) v / 2 = v / 2, i.e. a vector along v. The
+    # transposed readout R q = k (v.k) / 2 would point along k instead.
+    F, d = 20, 8
+    sizes = [2] + [0] * 4 + [1] + [0] * 4 + [3] * 10
+    inp = small_inputs(F, sizes=sizes, T=0, H=1, d=d, seed=31)
+    off = inp["off"]
+    k = inp["k"][off[5], 0].astype(np.float64)
+    v = inp["v"][off[5], 0].astype(np.float64)
+    row = int(off[17])                       # a token of frame 17 (block 3)
+    q = inp["q"].copy()
+    q[row, 0] = k
+    inp["q"] = q
+    res = O.layer_head(inp, 0, rows=np.array([row]))
+    # k is a float32 unit vector, so q . k_hat = ||k|| = 1 up to float32 rounding
+    np.testing.assert_allclose(res["o_lin"][0], np.linalg.norm(k) * v / 2, rtol=0, atol=1e-12)
+    cos_k = abs(res["o_lin"][0] @ k) / np.linalg.norm(res["o_lin"][0])
+    assert cos_k < 0.9  # not along k (k and v are independent draws)
+
+
+@pytest.mark.parametrize("F,seed", [(16, 41), (20, 42), (23, 43), (31, 44)])
+def test_both_scans_start_from_text_state_closed_form(F, seed):
+    # Every video key is the unit vector e1 and every video value is 0; frame
+    # f holds n_f in {0, 1, 2, 3} tokens. A frame update is then
+    # S -> (I + n e1 e1^T)^-1 S: row 0 of S is scaled by 1 / (1 + n) and the
+    # other rows are unchanged. Both scans start from S_text, so block b reads
+    #   R_b = 2 S_text with row 0 scaled by (a_f + a_b) / 2,
+    #   a_f = prod_{f=1..i_f} 1/(1+n_f),  a_b = prod_{f=i_b..F-2} 1/(1+n_f),
+    # with [w0, w1] = b's window, i_f = max(w0-1, 0), i_b = min(w1+1, F-1).
+    # A scan started from zero gives R_b = 0; a missing direction drops a term.
+    d = 6
+    rng = np.random.default_rng(seed)
+    sizes = rng.integers(0, 4, size=F)
+    inp = small_inputs(F, sizes=sizes, T=5, H=1, d=d, seed=seed)
+    k = np.zeros_like(inp["k"])
+    k[:, 0, 0] = 1.0
+    st = O.vda_states_head(k, np.zeros_like(inp["v"]), inp["kt"], inp["vt"],
+                           inp["off"], 0)
+    S_text = O.text_state(O.l2_normalise(inp["kt"][:, 0]), inp["vt"][:, 0], 1.0)
+    assert np.linalg.norm(S_text) > 0.1
+    for b in range(O.num_blocks(F)):
+        w0 = 5 * max(b - 1, 0)
+        w1 = min(5 * (b + 2), F) - 1
+        i_f, i_b = max(w0 - 1, 0), min(w1 + 1, F - 1)
+        a_f = np.prod([1.0 / (1 + sizes[f]) for f in range(1, i_f + 1)])
+        a_b = np.prod([1.0 / (1 + sizes[f]) for f in range(i_b, F - 1)])
+        ref = 2 * S_text
+        ref[0] = (a_f + a_b) * S_text[0]
+        np.testing.assert_allclose(st["R"][b], ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("F", [16, 20, 30])
+def test_text_values_reach_every_read_state(F):
+    # With F >= 16 at least one block reads scan states that have passed
+    # video frames; perturbing only the text values must still change every
+    # block's read state (the text initialises both scans).
+    inp = small_inputs(F, n=3, T=4, H=1, d=5, seed=F + 50)
+    a = O.vda_states_head(inp["k"], inp["v"], inp["kt"], inp["vt"], inp["off"], 0)
+    vt2 = inp["vt"] + 0.5 * np.random.default_rng(F).standard_normal(inp["vt"].shape)
+    b = O.vda_states_head(inp["k"], inp["v"], inp["kt"], vt2, inp["off"], 0)
+    assert any(i > 0 for i in (O.read_indices(bb, F)[0] for bb in range(O.num_blocks(F))))
+    for bb in range(O.num_blocks(F)):
+        assert np.linalg.norm(a["R"][bb] - b["R"][bb]) > 1e-6 * np.linalg.norm(a["R"][bb])

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <initializer_list>
+#include <mutex>
 
 #include "../../include/vdn.h"
 #include "k_audit.cuh"
@@ -556,36 +557,91 @@ const char* vdn_error_string(int code) {
 // ---------------------------------------------------------------------------
 // Linear-branch states without a caller-provided workspace.
 //
-// Some callers cannot hand this library a workspace: code that runs where
-// cudaMalloc is not allowed or not wanted (a host function enqueued with
-// cudaLaunchHostFunc may not call CUDA APIs that allocate; a serving loop
-// whose latency budget cannot absorb the implicit synchronisation of
-// cudaMalloc; a plug-in living inside a process whose memory is owned by
-// another allocator it has no handle to). For them, vdn_vda_scan_noalloc
-// keeps its scratch (per-frame C and W matrices, read-state halves and, for
-// fp32 or d < 128 inputs, the staged bf16 keys/values) in one file-scope
-// device array of kNoAllocScratchBytes. Every GPU that loads this library
-// holds that array until the process exits.
+// Some callers cannot hand this library a workspace: a serving loop whose
+// latency budget cannot absorb the implicit device synchronisation of
+// cudaMalloc / cudaFree, or a plug-in living inside a process whose device
+// memory is owned by another allocator it has no handle to. For them,
+// vdn_vda_scan_noalloc keeps its scratch (per-frame C and W matrices,
+// read-state halves and, for fp32 or d < 128 inputs, the staged bf16
+// keys/values) in one file-scope device array of kNoAllocScratchBytes. Every
+// GPU that loads this library holds that array until the process exits.
+// The entry point itself makes CUDA runtime calls and launches kernels, so
+// like every other entry point it must not be called from inside a stream
+// host function (cudaLaunchHostFunc callbacks may not call CUDA at all).
 // ---------------------------------------------------------------------------
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = (size_t)64 << 20;  // 64 MiB
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device. In host code
-// the symbol itself is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
-int noalloc_scratch_address(uint8_t** out) {
-  static uint8_t* addr[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return VDN_ERR_CUDA;
-  if (addr[dev] == nullptr) {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context (0 if there is none
+// yet). Context ids are never reused within a process, unlike device
+// ordinals (a context torn down by cudaDeviceReset and created again keeps
+// its ordinal but gets a new id and may map the array elsewhere).
+int current_context_id(unsigned long long* id) {
+  static const CtxGetCurrentFn get_cur = []() -> CtxGetCurrentFn {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return VDN_ERR_CUDA;
-    addr[dev] = static_cast<uint8_t*>(p);
+    cudaDriverEntryPointQueryResult q;
+    return (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+               ? reinterpret_cast<CtxGetCurrentFn>(p)
+               : nullptr;
+  }();
+  static const CtxGetIdFn get_id = []() -> CtxGetIdFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+               ? reinterpret_cast<CtxGetIdFn>(p)
+               : nullptr;
+  }();
+  if (get_cur == nullptr || get_id == nullptr) return VDN_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS) return VDN_ERR_CUDA;
+  *id = 0;
+  if (ctx != nullptr && get_id(ctx, id) != CUDA_SUCCESS) return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
+// Device address of g_noalloc_scratch in the current context. In host code
+// the symbol itself is only a host-side stand-in, so the address is looked up
+// with cudaGetSymbolAddress once per context (in practice once per device:
+// the runtime's primary context), with that device current, and cached under
+// the context's id. A mutex guards the cache against concurrent host threads.
+int noalloc_scratch_address(uint8_t** out) {
+  struct Entry {
+    unsigned long long ctx;
+    uint8_t* addr;
+  };
+  static std::mutex mu;
+  static Entry cache[64];
+  static int used = 0;
+  unsigned long long ctx = 0;
+  if (current_context_id(&ctx) != VDN_OK) return VDN_ERR_CUDA;
+  if (ctx != 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+      if (cache[i].ctx == ctx) {
+        *out = cache[i].addr;
+        return VDN_OK;
+      }
   }
-  *out = addr[dev];
+  // first call in this context (cudaGetSymbolAddress also creates the
+  // runtime's primary context if no context is current yet)
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return VDN_ERR_CUDA;
+  if (current_context_id(&ctx) != VDN_OK || ctx == 0) return VDN_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    bool found = false;
+    for (int i = 0; i < used && !found; ++i) found = (cache[i].ctx == ctx);
+    if (!found && used < 64) cache[used++] = Entry{ctx, static_cast<uint8_t*>(p)};
+  }
+  *out = static_cast<uint8_t*>(p);
   return VDN_OK;
 }
 
