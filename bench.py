@@ -1,13 +1,19 @@
 """Benchmark of the hybrid attention layer forward on B200.
 
 One step = one vdn_hybrid_attn_fwd call (softmax branch, VDA Grams/inverses,
-both scans, readout + RMSNorm + gated merge) on the pages-scale workload:
-F=15 latent frames of 24x42=1008 tokens (15120 video tokens), T=256 text
-tokens, H=32 heads, d=128, bf16, seed 0. Inputs are synthetic (vdn_synth).
+both scans, read-state packing, softmax kernel with the fused readout +
+RMSNorm + gated merge). The headline line runs the hi-res workload, the
+largest that fits one GPU: F=20 latent frames of 32x56=1792 tokens (35840
+video tokens), T=512 text tokens, H=24 heads, d=128, bf16, low-rank keys,
+seed 0. Inputs are synthetic (vdn_synth).
 
-Prints one JSON line (rank 0). `value` is layer TFLOP/s (algorithmic FLOP:
-softmax over unmasked (query, key) pairs + VDA Grams, inverses, scan products
-and readout) summed over ranks; `ms_per_step` is the max over ranks.
+Prints one JSON line (rank 0). `value` is layer TFLOP/s (algorithmic FLOP of
+the work the method needs: softmax over unmasked (query, key) pairs, VDA
+Grams / inverses / scan products of the frames some read state depends on,
+readout) summed over ranks; `ms_per_step` is the max over ranks. The line
+also carries `workloads`: ms/layer, TFLOP/s, per-kernel times and roofline
+fractions on every workload (the softmax kernel against the bf16 tensor peak,
+the VDA kernels and the standalone merge against HBM bandwidth).
 `--impl reference` times the fp64 CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
@@ -29,58 +35,102 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 
 METRIC = "hybrid-attn layer fwd ms and TFLOP/s (frac. of bf16 peak), 1×B200"
-WORKLOAD = "pages-scale"
-WORKLOAD_DESC = ("pages-scale single layer: F=15 latent frames (3 blocks of 5), 24x42=1008 "
-                 "tokens/frame (15120 video tokens), T=256 text tokens, H=32, d=128, bf16")
+HEADLINE = "hi-res"
+WORKLOADS = ["tiny", "pages-scale", "long-clip", "hi-res", "vda-stress"]
 L2_BYTES = 126 * 2 ** 20
+REF_ROWS = 2048          # query rows per reference-arm step (one head)
+CPU_BASELINE_HEADS = 12  # reference-arm steps in the GPU line's cpu_baseline
+
+
+# --------------------------------------------------------------- work model --
+
+def needed_frames(F: int, bf: int):
+    """Frames the read states depend on (the library skips the others when
+    no per-frame states are requested): the forward scan runs frames
+    1..fwd_last, the backward scan frames bwd_first..F-2; every needed frame
+    gets one Gram + inverse, each scan step one d x d x d product."""
+    fwd_last, bwd_first = 0, F - 1
+    for b in range(-(-F // bf)):
+        w0 = bf * max(b - 1, 0)
+        w1 = min(bf * (b + 2), F) - 1
+        fwd_last = max(fwd_last, max(w0 - 1, 0))
+        bwd_first = min(bwd_first, min(w1 + 1, F - 1))
+    frames = list(range(1, fwd_last + 1)) + list(range(max(bwd_first, fwd_last + 1), F - 1))
+    return dict(frames=frames, steps_fwd=1 + fwd_last, steps_bwd=1 + (F - 1 - bwd_first))
 
 
 def layer_flops(inp: dict, soft_pairs: np.ndarray) -> dict:
     """Algorithmic FLOP of one layer forward.
 
     softmax: 4 d H (video pairs + N T) over unmasked pairs (QK^T and PV);
-    VDA: Grams 4 (N+T) d^2 H, readout 2 N d^2 H, and per scanned matrix
-    (F-2 frames + text) and head one d x d inverse (2 d^3) plus one d^3 x 2
-    product per scan direction (4 d^3)."""
+    readout: 2 N d^2 H; VDA, over the text and the frames some read state
+    depends on: Grams 4 rows d^2 H (K^T K and K^T V), one d x d inverse per
+    matrix and head (2 d^3), one 2 d^3 product per scan step and head."""
     N, T, H, d, F = inp["N"], inp["T"], inp["H"], inp["d"], inp["F"]
+    off = np.asarray(inp["off"], np.int64)
+    nf = needed_frames(F, inp.get("block_frames", 5))
+    rows = T + sum(int(off[f + 1] - off[f]) for f in nf["frames"])
+    n_mat = 1 + len(nf["frames"])
     video_pairs = int(soft_pairs[:, :F].sum())
     softmax = 4.0 * d * H * (video_pairs + N * T)
-    grams = 4.0 * (N + T) * d * d * H
     readout = 2.0 * N * d * d * H
-    solves = (F - 1) * H * (2.0 * d ** 3 + 4.0 * d ** 3)
-    return dict(softmax=softmax, vda=grams + readout + solves,
-                total=softmax + grams + readout + solves)
+    grams = 4.0 * rows * d * d * H
+    inverses = 2.0 * d ** 3 * n_mat * H
+    scans = 2.0 * d ** 3 * (nf["steps_fwd"] + nf["steps_bwd"]) * H
+    vda = grams + inverses + scans
+    return dict(softmax=softmax, readout=readout, grams=grams, inverses=inverses, scans=scans,
+                vda=vda, total=softmax + readout + vda, gram_rows=rows, n_mat=n_mat,
+                scan_steps=nf["steps_fwd"] + nf["steps_bwd"])
 
 
-def vda_merge_roofline(inp: dict, layer_ms: float, softmax_ms: float, hbm_gbs: float) -> dict:
-    """VDA + merge path against its HBM roofline. Algorithmic bytes: k, v, kt,
-    vt read once, q, o_soft, g_s, g_l read and out written once (bf16). The
-    merge runs fused in the softmax kernel's epilogue, so the path's cost is
-    the layer time minus the softmax-only kernel."""
-    N, T, H, d = inp["N"], inp["T"], inp["H"], inp["d"]
-    act = N * H * d * 2
-    nbytes = 2 * act + 2 * T * H * d * 2 + 2 * act + 2 * N * H * 2 + act
-    roof_ms = nbytes / (hbm_gbs * 1e9) * 1e3
-    marginal = layer_ms - softmax_ms
-    return {"algorithmic_bytes": int(nbytes), "roofline_ms": round(roof_ms, 4),
-            "marginal_ms": round(marginal, 4),
-            "frac": round(roof_ms / marginal, 4) if marginal > 0 else None,
-            "method": "layer time minus the softmax-only kernel (merge fused in its epilogue)"}
+def kernel_bytes(inp: dict, fl: dict) -> dict:
+    """Algorithmic HBM bytes per launch of the HBM-bound kernels (d = 128 bf16):
+    Gram + inverse reads k, v of its rows once and writes C and W once; a scan
+    step reads W_f and C_f once and the scans write the two read-state halves;
+    packing reads both halves and writes one bf16 tile per (block, head); the
+    standalone readout + merge reads q, o_soft, gates and R_b and writes out."""
+    N, T, H, d, F = inp["N"], inp["T"], inp["H"], inp["d"], inp["F"]
+    nb = -(-F // inp["block_frames"])
+    mat = 128 * 128 * 4
+    return dict(
+        gram_inv=2 * fl["gram_rows"] * H * d * 2 + 2 * fl["n_mat"] * H * mat,
+        scan=fl["scan_steps"] * H * 2 * mat + 2 * nb * H * mat,
+        pack=2 * nb * H * mat + nb * H * 128 * 128 * 2,
+        gate_merge=3 * N * H * d * 2 + 2 * N * H * 2 + nb * H * d * d * 4,
+    )
 
 
 def workload_desc(name: str) -> str:
-    if name == WORKLOAD:
-        return WORKLOAD_DESC
     import vdn_synth as S
     c = S.CONFIGS[name]
+    extra = ""
+    if c.get("k_lowrank"):
+        extra = f", keys rank {c['k_lowrank']} + 0.1 noise per frame"
+    if c.get("short_every"):
+        extra = (f", frames f%{c['short_every']}=={c['short_every'] - 1} hold {c['short_n']} "
+                 f"tokens, frames f%{c['zero_v_every']}=={c['zero_v_every'] - 1} have v=0")
     return (f"{name}: F={c['F']} latent frames, {c['grid'][0]}x{c['grid'][1]} tokens/frame, "
-            f"T={c['T']}, H={c['H']}, d={c['d']}, {c['dtype']}")
+            f"T={c['T']}, H={c['H']}, d={c['d']}, {c['dtype']}{extra}")
 
 
-def l2_note(input_bytes: int) -> str:
-    if input_bytes > L2_BYTES:
-        return f"inputs {input_bytes / 2 ** 20:.0f} MiB > 126 MB L2; no flush between steps"
-    return "inputs fit in the 126 MB L2: warm-cache figure, no flush between steps"
+def input_bytes(inp: dict) -> int:
+    e = 2 if inp["dtype"] == "bf16" else 4
+    return (3 * inp["N"] + 2 * inp["T"]) * inp["H"] * inp["d"] * e + 2 * inp["N"] * inp["H"] * e
+
+
+def l2_note(nbytes: int) -> str:
+    if nbytes > L2_BYTES:
+        return f"inputs {nbytes / 2 ** 20:.0f} MiB > 126 MB L2; no flush between steps"
+    return "inputs fit in the 126 MB L2: L2 flushed (256 MiB write) before every timed step"
+
+
+def config_of(name: str, inp: dict, fl: dict, world: int) -> dict:
+    """The `config` object, identical for the CUDA and the reference arm."""
+    return {"workload": workload_desc(name), "F": inp["F"],
+            "tokens_per_frame": int(inp["N"] // inp["F"]), "N": inp["N"], "T": inp["T"],
+            "H": inp["H"], "d": inp["d"], "layer_tflop": round(fl["total"] / 1e12, 4),
+            "softmax_tflop": round(fl["softmax"] / 1e12, 4),
+            "parallelism": f"replicas x{world}", "l2": l2_note(input_bytes(inp))}
 
 
 def load_peaks() -> dict:
@@ -88,9 +138,10 @@ def load_peaks() -> dict:
     if os.path.exists(path):
         with open(path) as fh:
             p = json.load(fh)
-        return dict(bf16_tflops=float(p["bf16_tflops"]), hbm_gbs=float(p["hbm_gbs"]),
-                    source="measured")
-    return dict(bf16_tflops=1590.0, hbm_gbs=6650.0, source="fallback")
+        return dict(bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    hbm_gbs=float(p["hbm_gbs"]), source="measured")
+    return dict(bf16_tflops=1590.0, bf16_sustained=1400.0, hbm_gbs=6650.0, source="fallback")
 
 
 def bsa_source_hash() -> str:
@@ -101,21 +152,21 @@ def bsa_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic():
-    """DRAM bytes per k_bsa_fwd launch from the committed ncu summary, if it
-    was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "bsa_fwd_pages_scale_traffic.json")
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the merged softmax kernel from the committed
+    ncu summary, if it was taken on the current kernel source and workload."""
+    path = os.path.join(ROOT, "profiles", "bsa_fwd_merge_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as fh:
         rec = json.load(fh)
-    if rec.get("source_hash") != bsa_source_hash():
+    if rec.get("source_hash") != bsa_source_hash() or rec.get("workload") != workload:
         return None
     return rec.get("dram_bytes_per_launch")
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms (read only)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -191,11 +242,148 @@ def dist_env():
     return world, rank, local
 
 
+def cores_used() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------- CUDA arm -----
+
+class Workload:
+    """One workload's inputs on the device plus the buffers the entry points need."""
+
+    def __init__(self, name: str, V, torch):
+        import vdn_synth as S
+        self.name = name
+        self.inp = inp = S.make_inputs(name, seed=0)
+        self.dt = torch.bfloat16 if inp["dtype"] == "bf16" else torch.float32
+        self.host = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to(self.dt)
+                     for k in ("q", "k", "v", "kt", "vt", "g_s", "g_l")}
+        self.dev = {k: t.to("cuda") for k, t in self.host.items()}
+        self.rms_w = torch.from_numpy(inp["rms_w"]).cuda()
+        self.shape = V.Shape(inp["off"], inp["T"], inp["H"], inp["d"], inp["block_frames"],
+                             inp["lam"], inp["eps"],
+                             V.VDN_BF16 if inp["dtype"] == "bf16" else V.VDN_F32)
+        self.ws = V.alloc_workspace(self.shape)
+        self.out = torch.empty_like(self.dev["q"])
+        soft = torch.empty((inp["F"], inp["F"] + 1), dtype=torch.int64, device="cuda")
+        lin = torch.empty((inp["F"], inp["F"]), dtype=torch.int64, device="cuda")
+        V.vdn_pair_audit(self.shape, soft, lin)
+        self.fl = layer_flops(inp, soft.cpu().numpy())
+        self.bytes = kernel_bytes(inp, self.fl)
+        self.flush = input_bytes(inp) <= L2_BYTES
+
+    def layer(self, V, stream, dev=None, out=None):
+        d = dev or self.dev
+        V.vdn_hybrid_attn_fwd(self.shape, d["q"], d["k"], d["v"], d["kt"], d["vt"], d["g_s"],
+                              d["g_l"], self.rms_w, out if out is not None else self.out, self.ws,
+                              stream)
+
+
+def time_launches(torch, stream, fn, n: int, flush=None) -> float:
+    """Mean ms of `fn` over n launches, CUDA events on `stream`. With `flush`
+    (a >L2 buffer), each launch is timed alone after overwriting L2."""
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+    tot = 0.0
+    for _ in range(n):
+        flush.add_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    return tot / n
+
+
+def workload_report(V, torch, w: Workload, stream, steps: int, warmup: int, peaks: dict,
+                    flush_buf) -> dict:
+    """ms/layer, TFLOP/s and per-kernel roofline fractions of one workload."""
+    for _ in range(warmup):
+        w.layer(V, stream)
+    torch.cuda.synchronize()
+    rc = V.vdn_get_device_error()
+    if rc != 0:
+        raise RuntimeError(f"{w.name}: {V.vdn_error_string(rc)}")
+    fb = flush_buf if w.flush else None
+    ms = time_launches(torch, stream, lambda: w.layer(V, stream), steps, fb)
+    kern = V.vdn_hybrid_attn_fwd_profile(w.shape, w.dev["q"], w.dev["k"], w.dev["v"],
+                                         w.dev["kt"], w.dev["vt"], w.dev["g_s"], w.dev["g_l"],
+                                         w.rms_w, w.out, w.ws, iters=min(steps, 20),
+                                         stream=stream)
+    fl = w.fl
+    merged_flop = fl["softmax"] + fl["readout"]
+    t_sm = kern["softmax_merge"]
+    rep = {
+        "ms_per_layer": round(ms, 4),
+        "tflops": round(fl["total"] / (ms * 1e-3) / 1e12, 1),
+        "layer_tflop": round(fl["total"] / 1e12, 4),
+        "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
+        "softmax_merge": {
+            "kernel": "k_bsa_fwd<merge>", "flop": merged_flop,
+            "achieved_tflops": round(merged_flop / (t_sm * 1e-3) / 1e12, 1),
+            "frac_burst": round(merged_flop / (t_sm * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "frac_sustained": round(merged_flop / (t_sm * 1e-3) / 1e12 / peaks["bf16_sustained"], 4),
+        },
+    }
+    if w.inp["d"] == 128 and w.inp["dtype"] == "bf16":
+        # softmax branch alone (no merge epilogue), and the standalone merge
+        o_soft = torch.empty(w.dev["q"].shape, dtype=torch.bfloat16, device="cuda")
+        nb = w.shape.nb
+        R = torch.empty((nb, w.inp["H"], 128, 128), device="cuda")
+        d = w.dev
+        V.vdn_vda_scan(w.shape, d["k"], d["v"], d["kt"], d["vt"], R, None, None, None, w.ws,
+                       stream)
+
+        def bsa():
+            V.vdn_bsa_fwd(w.shape, d["q"], d["k"], d["v"], d["kt"], d["vt"], o_soft, None, w.ws,
+                          stream)
+
+        def merge():
+            V.vdn_gate_merge(w.shape, d["q"], R, o_soft, d["g_s"], d["g_l"], w.rms_w, w.out, w.ws,
+                             stream)
+
+        bsa()
+        t_bsa = time_launches(torch, stream, bsa, max(3, steps // 2))
+        merge()
+        t_merge = time_launches(torch, stream, merge, max(5, steps))
+        rep["softmax_only"] = {"kernel": "k_bsa_fwd", "ms": round(t_bsa, 4),
+                               "frac_burst": round(fl["softmax"] / (t_bsa * 1e-3) / 1e12
+                                                   / peaks["bf16_tflops"], 4)}
+        hbm = {}
+        for key, t in (("gram_inv", kern["gram_inv"]), ("scan", kern["scan"]),
+                       ("pack", kern["pack"]), ("gate_merge", t_merge)):
+            b = w.bytes[key]
+            gbs = b / (t * 1e-3) / 1e9 if t > 0 else None
+            hbm[key] = {"bytes": int(b), "ms": round(t, 4),
+                        "gbs": round(gbs, 1) if gbs else None,
+                        "frac": round(gbs / peaks["hbm_gbs"], 4) if gbs else None}
+        hbm["gate_merge"]["kernel"] = "k_readout_merge_tma (vdn_gate_merge)"
+        rep["hbm"] = hbm
+        del o_soft, R
+    # outputs are still valid after the helper runs (same computation)
+    torch.cuda.synchronize()
+    rc = V.vdn_get_device_error()
+    if rc != 0:
+        raise RuntimeError(f"{w.name}: {V.vdn_error_string(rc)}")
+    return rep
+
+
 def run_cuda(args) -> None:
     import torch
 
     import video_diffusion_hybrid_block_b200 as V
-    import vdn_synth as S
 
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -205,82 +393,52 @@ def run_cuda(args) -> None:
 
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-    inp = S.make_inputs(args.workload, seed=0)
-    dt = torch.bfloat16 if inp["dtype"] == "bf16" else torch.float32
-    host = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to(dt).pin_memory()
-            for k in ("q", "k", "v", "kt", "vt", "g_s", "g_l")}
-    dev = {k: t.to("cuda", non_blocking=False) for k, t in host.items()}
-    rms_w = torch.from_numpy(inp["rms_w"]).cuda()
-    shape = V.Shape(inp["off"], inp["T"], inp["H"], inp["d"], inp["block_frames"], inp["lam"],
-                    inp["eps"], V.VDN_BF16 if inp["dtype"] == "bf16" else V.VDN_F32)
-    ws = V.alloc_workspace(shape)
-    out = torch.empty_like(dev["q"])
-    out_host = torch.empty(out.shape, dtype=dt).pin_memory()
     stream = torch.cuda.current_stream()
-
-    soft = torch.empty((inp["F"], inp["F"] + 1), dtype=torch.int64, device="cuda")
-    lin = torch.empty((inp["F"], inp["F"]), dtype=torch.int64, device="cuda")
-    V.vdn_pair_audit(shape, soft, lin)
-    fl = layer_flops(inp, soft.cpu().numpy())
-
-    def step():
-        V.vdn_hybrid_attn_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"],
-                              dev["g_s"], dev["g_l"], rms_w, out, ws, stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    rc = V.vdn_get_device_error()
-    if rc != 0:
-        raise RuntimeError(V.vdn_error_string(rc))
+    peaks = load_peaks()
 
     def barrier():
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize()
 
-    # ---- device-resident timing of the whole layer
+    # ---- headline workload: device-resident timing of the whole layer
+    w = Workload(args.workload, V, torch)
+    for _ in range(args.warmup):
+        w.layer(V, stream)
+    torch.cuda.synchronize()
+    rc = V.vdn_get_device_error()
+    if rc != 0:
+        raise RuntimeError(V.vdn_error_string(rc))
+    flush_buf = torch.empty(64 * 2 ** 20, dtype=torch.float32, device="cuda")  # 256 MiB
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        barrier()
-    ms = max_over_ranks(dist, e0.elapsed_time(e1) / args.steps, "cuda")
+        if w.flush:
+            barrier()
+            ms = time_launches(torch, stream, lambda: w.layer(V, stream), args.steps, flush_buf)
+            barrier()
+        else:
+            barrier()
+            e0.record(stream)
+            for _ in range(args.steps):
+                w.layer(V, stream)
+            e1.record(stream)
+            barrier()
+            ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(dist, ms, "cuda")
     clocks = clk.summary()
-    launches_per_step = 4 + (0 if shape.d == 128 else 5)
-
-    # ---- dominant kernel alone (softmax branch), CUDA events on its stream
-    o_soft = torch.empty(dev["q"].shape, dtype=torch.bfloat16, device="cuda")
-
-    def bsa():
-        V.vdn_bsa_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"], o_soft, None,
-                      ws, stream)
-
-    for _ in range(3):
-        bsa()
-    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    b0.record(stream)
-    nb_launch = max(args.steps, 5)
-    for _ in range(nb_launch):
-        bsa()
-    b1.record(stream)
-    barrier()
-    bsa_ms = max_over_ranks(dist, b0.elapsed_time(b1) / nb_launch, "cuda")
+    launches_per_step = 4 + (0 if (w.inp["d"] == 128 and w.inp["dtype"] == "bf16") else 5)
 
     # ---- end to end through the C ABI with host buffers (H2D + layer + D2H).
     # Every step copies its inputs from pinned host memory and its output back.
     # Two device buffer sets let step i+1's upload (copy stream) run while step
     # i computes and step i-1's result downloads (second copy stream), as a
     # serving loop would; each step still moves all of its bytes.
+    host = {k: t.pin_memory() for k, t in w.host.items()}
+    out_host = torch.empty(w.out.shape, dtype=w.dt).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out.numel() * out.element_size()
-    sets = [dev, {k: torch.empty_like(t) for k, t in dev.items()}]
-    outs = [out, torch.empty_like(out)]
+    d2h = w.out.numel() * w.out.element_size()
+    sets = [w.dev, {k: torch.empty_like(t) for k, t in w.dev.items()}]
+    outs = [w.out, torch.empty_like(w.out)]
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev = {n: [torch.cuda.Event(), torch.cuda.Event()] for n in ("up", "done", "down")}
     for b in range(2):  # all buffers free at the start
@@ -297,8 +455,7 @@ def run_cuda(args) -> None:
             ev["up"][b].record(s_in)
         stream.wait_event(ev["up"][b])
         stream.wait_event(ev["down"][b])     # out b was downloaded
-        V.vdn_hybrid_attn_fwd(shape, d["q"], d["k"], d["v"], d["kt"], d["vt"], d["g_s"], d["g_l"],
-                              rms_w, o, ws, stream)
+        w.layer(V, stream, dev=d, out=o)
         ev["done"][b].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev["done"][b])
@@ -317,10 +474,22 @@ def run_cuda(args) -> None:
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(dist, g0.elapsed_time(g1) / args.steps, "cuda")
+    del sets[1], outs[1]
 
-    peaks = load_peaks()
-    achieved = fl["softmax"] / (bsa_ms * 1e-3) / 1e12
-    value = whole_job_value(world, fl["total"], ms)
+    # ---- every workload (the headline's object is measured on its buffers)
+    reports = {}
+    names = [args.workload] if args.workloads == "none" else WORKLOADS
+    for name in names:
+        ww = w if name == args.workload else Workload(name, V, torch)
+        reports[name] = workload_report(V, torch, ww, stream, args.steps, args.warmup, peaks,
+                                        flush_buf)
+        if ww is not w:
+            del ww
+            torch.cuda.empty_cache()
+    head = reports[args.workload]
+    sm = head["softmax_merge"]
+
+    value = whole_job_value(world, w.fl["total"], ms)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -334,29 +503,27 @@ def run_cuda(args) -> None:
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": workload_desc(args.workload), "F": inp["F"],
-                   "tokens_per_frame": int(inp["N"] // inp["F"]),
-                   "N": inp["N"], "T": inp["T"], "H": inp["H"], "d": inp["d"],
-                   "layer_tflop": round(fl["total"] / 1e12, 4),
-                   "softmax_tflop": round(fl["softmax"] / 1e12, 4),
-                   "parallelism": f"replicas x{world}", "l2": l2_note(h2d)},
-        "roofline": {"kernel": "k_bsa_fwd", "bound": "tensor", "achieved": round(achieved, 1),
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(achieved / peaks["bf16_tflops"], 4),
-                     "peak_source": f"{peaks['source']} bf16 burst",
-                     "launch_ms": round(bsa_ms, 4),
-                     "traffic": recorded_traffic() if args.workload == WORKLOAD else None},
-        "e2e": {"value": round(whole_job_value(world, fl["total"], e2e_ms), 2),
+        "config": config_of(args.workload, w.inp, w.fl, world),
+        "roofline": {"kernel": "k_bsa_fwd<merge> (softmax branch + fused readout, RMSNorm, "
+                               "gated merge), timed inside the layer",
+                     "bound": "tensor", "achieved": sm["achieved_tflops"],
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": sm["frac_burst"],
+                     "frac_sustained": sm["frac_sustained"],
+                     "peak_source": f"{peaks['source']} bf16 burst "
+                                    f"(sustained {peaks['bf16_sustained']})",
+                     "launch_ms": head["kernels_ms"]["softmax_merge"],
+                     "traffic": recorded_traffic(args.workload)},
+        "e2e": {"value": round(whole_job_value(world, w.fl["total"], e2e_ms), 2),
                 "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "pipelining": "uploads, layer and downloads of consecutive steps overlap "
                               "(two device buffer sets, two copy streams)",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
-        "vda_merge": vda_merge_roofline(inp, ms, bsa_ms, peaks["hbm_gbs"]),
+        "workloads": reports,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
-        line["cpu_baseline"] = cpu_baseline(inp, fl, args.cpu_heads)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w.inp, w.fl, args.workload, CPU_BASELINE_HEADS)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -364,25 +531,81 @@ def run_cuda(args) -> None:
         print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(inp: dict, fl: dict, heads: int) -> dict:
-    """The fp64 CPU oracle, as it stands, on `heads` of the workload's heads
-    (every query row of those heads); scaled to the layer's FLOP per head."""
-    import oracle as O
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count()
-    t0 = time.perf_counter()
-    for h in range(heads):
-        O.layer_head(inp, h)
-    dt = time.perf_counter() - t0
-    flop = fl["total"] * heads / inp["H"]
-    return {"value": round(flop / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
-            "kind": "oracle", "seconds": round(dt, 2),
-            "sample": f"fp64 numpy oracle, whole layer for {heads} of {inp['H']} heads "
-                      f"(all {inp['N']} query rows), pages-scale workload"}
+# --------------------------------------------------------- oracle (CPU) -----
 
+def reference_rows(inp: dict, n: int = REF_ROWS) -> np.ndarray:
+    """Query rows one reference step computes: n rows evenly spread over the clip."""
+    return np.unique(np.linspace(0, inp["N"] - 1, min(n, inp["N"])).astype(np.int64))
+
+
+def reference_step_flops(inp: dict, soft_pairs: np.ndarray, fl: dict, rows) -> float:
+    """Algorithmic FLOP of one reference step: one head's VDA work plus the
+    softmax and readout work of the given query rows of that head."""
+    off = np.asarray(inp["off"], np.int64)
+    F, d, H, T = inp["F"], inp["d"], inp["H"], inp["T"]
+    n = np.diff(off)
+    keys = np.where(n > 0, soft_pairs[:, :F].sum(axis=1) / np.maximum(n, 1), 0) + T
+    frame = np.searchsorted(off, rows, side="right") - 1
+    return fl["vda"] / H + 4.0 * d * float(keys[frame].sum()) + 2.0 * d * d * len(rows)
+
+
+def oracle_steps(inp: dict, fl: dict, soft: np.ndarray, nsteps: int, warmup: int):
+    """Runs the fp64 oracle as it stands: step s = head s % H, all of its VDA
+    states and the whole layer for REF_ROWS query rows. Returns (seconds per
+    step, FLOP per step)."""
+    import oracle as O
+    rows = reference_rows(inp)
+    for s in range(warmup):
+        O.layer_head(inp, s % inp["H"], rows=rows)
+    t0 = time.perf_counter()
+    for s in range(nsteps):
+        O.layer_head(inp, s % inp["H"], rows=rows)
+    dt = (time.perf_counter() - t0) / max(nsteps, 1)
+    return dt, reference_step_flops(inp, soft, fl, rows)
+
+
+def cpu_baseline(inp: dict, fl: dict, name: str, heads: int) -> dict:
+    """The fp64 CPU oracle, as it stands, on a bounded sample of the workload."""
+    import oracle as O
+    soft, _ = O.pair_counts(inp["off"], inp["block_frames"], inp["T"])
+    dt, flop = oracle_steps(inp, fl, soft, heads, 0)
+    return {"value": round(flop / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores_used(),
+            "kind": "oracle", "seconds": round(dt * heads, 2),
+            "sample": f"fp64 numpy oracle, {heads} heads of {inp['H']}: each head's VDA states "
+                      f"and the whole layer for {len(reference_rows(inp))} of {inp['N']} query "
+                      f"rows, {name} workload"}
+
+
+def run_reference(args) -> None:
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle as O
+    import vdn_synth as S
+    inp = S.make_inputs(args.workload, seed=0)
+    soft, _ = O.pair_counts(inp["off"], inp["block_frames"], inp["T"])
+    fl = layer_flops(inp, soft)
+    dt, flop = oracle_steps(inp, fl, soft, args.steps, args.warmup)
+    value = flop / dt / 1e12
+    rows = reference_rows(inp)
+    sample = (f"fp64 numpy oracle; one step = one head's VDA states and the whole layer for "
+              f"{len(rows)} of {inp['N']} query rows, {args.workload} workload")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(args.workload, inp, fl, world),
+        "step_tflop": round(flop / 1e12, 6),
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores_used(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ ncu helper ----
 
 def run_profile(args) -> None:
     """Runs `--steps` launches of one entry point (after `--warmup`) on a
@@ -437,58 +660,18 @@ def run_profile(args) -> None:
         sys.exit(1)
 
 
-def run_reference(args) -> None:
-    world, rank, _ = dist_env()
-    if rank != 0:
-        return
-    import vdn_synth as S
-    import oracle as O
-    inp = S.make_inputs(WORKLOAD, seed=0)
-    soft, _ = O.pair_counts(inp["off"], inp["block_frames"], inp["T"])
-    fl = layer_flops(inp, soft)
-    for _ in range(args.warmup):
-        O.layer_head(inp, 0)
-    times = []
-    for s in range(args.steps):
-        t0 = time.perf_counter()
-        O.layer_head(inp, s % inp["H"])
-        times.append(time.perf_counter() - t0)
-    per_head = sum(times) / len(times)
-    flop = fl["total"] / inp["H"]
-    value = flop / per_head / 1e12
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count()
-    sample = (f"fp64 numpy oracle, one head (all {inp['N']} query rows) per step, "
-              "pages-scale workload")
-    line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(per_head * 1e3 * inp["H"], 1), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESC, "F": inp["F"], "N": inp["N"], "T": inp["T"],
-                   "H": inp["H"], "d": inp["d"], "parallelism": "cpu"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
-                         "kind": "oracle", "sample": sample},
-        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-
-
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--cpu-heads", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default="all", choices=["all", "none"],
+                    help="also report every workload (default) or only the headline one")
     ap.add_argument("--profile", choices=["layer", "bsa", "vda", "merge"],
                     help="only run launches of one entry point (for ncu captures)")
-    ap.add_argument("--workload", default=WORKLOAD,
+    ap.add_argument("--workload", default=HEADLINE,
                     help="workload name (vdn_synth.CONFIGS); the default is the headline one")
     ap.add_argument("--heads", type=int, default=0, help="override head count for --profile")
     args = ap.parse_args()

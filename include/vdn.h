@@ -109,6 +109,23 @@ int vdn_hybrid_attn_fwd(const vdn_shape_t* shape, const void* q, const void* k,
                         const void* g_s, const void* g_l, const float* rms_w,
                         void* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* Measurement helper (no paper counterpart). Runs vdn_hybrid_attn_fwd (same
+ * arguments) `iters` times (1..256) on `stream` with CUDA events recorded on
+ * that stream between its kernels, waits for the stream, and writes the mean
+ * time per layer, in ms, of each launch group to kernel_ms[5]:
+ *   [0] fp32 narrowing / head-dim padding (about 0 when not needed),
+ *   [1] Gram matrices + inverses, [2] forward/backward scans,
+ *   [3] read-state packing, [4] softmax branch with the fused readout,
+ *   RMSNorm and gated merge.
+ * Unlike every other entry point it synchronises the stream and creates and
+ * destroys its own events (host-side only; no device memory is allocated).
+ * The event records add a few microseconds between kernels. */
+int vdn_hybrid_attn_fwd_profile(const vdn_shape_t* shape, const void* q, const void* k,
+                                const void* v, const void* kt, const void* vt,
+                                const void* g_s, const void* g_l, const float* rms_w,
+                                void* out, void* workspace, size_t ws_bytes, void* stream,
+                                int iters, float* kernel_ms);
+
 /* Linear branch states only. read_states [nb, H, d, d] fp32 (required;
  * nb = ceil(F / block_frames)) gets R_b. Optional (NULL to skip):
  * text_state [H, d, d]; fwd_states [F, H, d, d] gets Sfwd[i] for

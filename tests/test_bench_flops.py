@@ -32,10 +32,10 @@ def brute_softmax_pairs(off, bf, T):
 def test_softmax_flop_count_matches_brute_force(sizes, bf, T):
     off = S.frame_offsets(sizes)
     soft, _ = O.pair_counts(off, bf, T)
-    inp = dict(N=int(off[-1]), T=T, H=3, d=32, F=len(sizes))
+    inp = dict(N=int(off[-1]), T=T, H=3, d=32, F=len(sizes), off=off, block_frames=bf)
     fl = bench.layer_flops(inp, soft)
     assert fl["softmax"] == 4.0 * 32 * 3 * brute_softmax_pairs(off, bf, T)
-    assert fl["total"] == fl["softmax"] + fl["vda"]
+    assert fl["total"] == fl["softmax"] + fl["readout"] + fl["vda"]
 
 
 def test_pages_scale_softmax_flop():
@@ -55,10 +55,58 @@ def test_workload_descriptions_and_l2_notes():
     assert "fit in the 126 MB L2" in bench.l2_note(2 ** 20)
 
 
-def test_vda_merge_roofline_bytes():
-    # 625.7 MB at pages-scale: k, v, q, o_soft, out 124 MB each, kt, vt, gates
+@pytest.mark.parametrize("F,bf", [(2, 5), (10, 5), (11, 5), (15, 5), (20, 5), (30, 5), (60, 5),
+                                  (9, 1), (30, 7), (14, 3)])
+def test_needed_frames_are_the_linear_frames_of_some_block(F, bf):
+    # the frames whose Grams/inverses the library computes are exactly the
+    # frames some block folds into its read state (oracle's linear key frames)
+    nf = bench.needed_frames(F, bf)
+    want = sorted(set().union(*[O.linear_key_frames(b, F, bf) for b in range(O.num_blocks(F, bf))]))
+    assert nf["frames"] == want
+    i_f = [O.read_indices(b, F, bf)[0] for b in range(O.num_blocks(F, bf))]
+    i_b = [O.read_indices(b, F, bf)[1] for b in range(O.num_blocks(F, bf))]
+    assert nf["steps_fwd"] == 1 + max(i_f)
+    assert nf["steps_bwd"] == 1 + (F - 1 - min(i_b))
+
+
+def test_pages_scale_vda_counts_and_kernel_bytes():
+    # pages-scale: 8 of 13 scanned frames are needed (1..4 and 10..13), 5 scan
+    # steps per direction; the Gram kernel reads 136.3 MB of k, v and writes
+    # 37.7 MB of C and W
     inp = S.make_inputs("pages-scale")
-    r = bench.vda_merge_roofline(inp, 2.766, 2.640, 6543.0)
-    assert r["algorithmic_bytes"] == 5 * 15120 * 32 * 128 * 2 + 2 * 256 * 32 * 128 * 2 + 2 * 15120 * 32 * 2
-    assert abs(r["roofline_ms"] - r["algorithmic_bytes"] / 6543e9 * 1e3) < 1e-4
-    assert abs(r["marginal_ms"] - 0.126) < 1e-9 and abs(r["frac"] - r["roofline_ms"] / 0.126) < 1e-3
+    soft, _ = O.pair_counts(inp["off"], 5, inp["T"])
+    fl = bench.layer_flops(inp, soft)
+    assert fl["n_mat"] == 9 and fl["scan_steps"] == 10
+    assert fl["gram_rows"] == 256 + 8 * 1008
+    assert fl["grams"] == 4.0 * (256 + 8 * 1008) * 128 ** 2 * 32
+    kb = bench.kernel_bytes(inp, fl)
+    assert kb["gram_inv"] == 2 * 8320 * 32 * 128 * 2 + 2 * 9 * 32 * 65536
+    assert kb["gate_merge"] == 3 * 15120 * 32 * 128 * 2 + 2 * 15120 * 32 * 2 + 3 * 32 * 65536
+    assert fl["total"] == fl["softmax"] + fl["readout"] + fl["vda"]
+
+
+def test_reference_step_flops_brute_force():
+    # one head's VDA work + 4 d |J(i)| per sampled row + 2 d^2 per row
+    sizes = [7, 3, 0, 5, 9, 2, 4, 6, 1, 8, 3, 5]
+    off = S.frame_offsets(sizes)
+    T, d, H = 4, 32, 3
+    soft, _ = O.pair_counts(off, 5, T)
+    inp = dict(N=int(off[-1]), T=T, H=H, d=d, F=len(sizes), off=off, block_frames=5)
+    fl = bench.layer_flops(inp, soft)
+    rows = np.array([0, 6, 7, 20, 30, 52])
+    frame = np.repeat(np.arange(len(sizes)), sizes)
+    keys = 0
+    for i in rows:
+        allowed = set(O.softmax_key_frames(O.block_of(int(frame[i])), len(sizes)))
+        keys += int(np.isin(frame, list(allowed)).sum()) + T
+    want = fl["vda"] / H + 4.0 * d * keys + 2.0 * d * d * len(rows)
+    assert bench.reference_step_flops(inp, soft, fl, rows) == pytest.approx(want, rel=1e-12)
+
+
+def test_config_is_shared_by_both_arms():
+    inp = S.make_inputs("tiny")
+    soft, _ = O.pair_counts(inp["off"], 5, inp["T"])
+    fl = bench.layer_flops(inp, soft)
+    a = bench.config_of("tiny", inp, fl, 1)
+    assert set(a) >= {"workload", "F", "N", "T", "H", "d", "parallelism", "l2"}
+    assert "fit in the 126 MB L2" in a["l2"]

@@ -264,3 +264,23 @@ def test_gate_merge_entry_matches_layer(d):
         oref = O.layer_head(inp, h)["out"]
         assert rel_l2(got[:, h], oref) <= OUT_REL_L2, h
         assert max_abs(got[:, h], oref) <= OUT_MAX_ABS, h
+
+
+def test_profile_entry_matches_layer():
+    # the measurement helper runs the same launches: identical output, and a
+    # positive time for every kernel group the bf16 d = 128 layer launches
+    import video_diffusion_hybrid_block_b200 as V
+    from vdn_cases import make_shape
+    inp = mid_case(seed=9)
+    dev = device_inputs(inp)
+    ref = run_layer(inp, dev)
+    shape = make_shape(inp)
+    ws = V.alloc_workspace(shape)
+    out = torch.empty_like(dev["q"])
+    ms = V.vdn_hybrid_attn_fwd_profile(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"],
+                                       dev["g_s"], dev["g_l"], dev["rms_w"], out, ws, iters=3)
+    assert V.vdn_get_device_error() == 0
+    assert torch.equal(out, ref)
+    assert set(ms) == set(V.PROFILE_GROUPS)
+    for k in ("gram_inv", "scan", "pack", "softmax_merge"):
+        assert ms[k] > 0, k

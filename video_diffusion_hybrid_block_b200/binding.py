@@ -55,6 +55,8 @@ _SZ = ctypes.c_size_t
 _SIGS = {
     "vdn_workspace_bytes": (_SZ, [ctypes.POINTER(vdn_shape_t)]),
     "vdn_hybrid_attn_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 9 + [_P, _SZ, _P]),
+    "vdn_hybrid_attn_fwd_profile": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 9
+                                    + [_P, _SZ, _P, ctypes.c_int, ctypes.POINTER(ctypes.c_float)]),
     "vdn_vda_scan": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 8 + [_P, _SZ, _P]),
     "vdn_gate_merge": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
     "vdn_bsa_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
@@ -193,6 +195,25 @@ def vdn_hybrid_attn_fwd(shape: Shape, q, k, v, kt, vt, g_s, g_l, rms_w, out, wor
         _stream(stream))
     _check(rc, "vdn_hybrid_attn_fwd")
     return out
+
+
+PROFILE_GROUPS = ("stage", "gram_inv", "scan", "pack", "softmax_merge")
+
+
+def vdn_hybrid_attn_fwd_profile(shape: Shape, q, k, v, kt, vt, g_s, g_l, rms_w, out, workspace,
+                                iters: int = 10, stream=None, ws_bytes=None) -> dict:
+    """Runs the layer `iters` times with CUDA events between its kernels and
+    returns the mean ms per layer of each launch group (PROFILE_GROUPS).
+    Synchronises the stream (measurement helper)."""
+    _check_acts(shape, q, k, v, kt, vt, g_s, g_l, out)
+    _need(rms_w, shape.H * shape.d, 4, "rms_w")
+    ms = (ctypes.c_float * len(PROFILE_GROUPS))()
+    rc = load_library().vdn_hybrid_attn_fwd_profile(
+        shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(g_s), _ptr(g_l),
+        _ptr(rms_w), _ptr(out), _ptr(workspace), _nbytes(workspace, ws_bytes),
+        _stream(stream), int(iters), ms)
+    _check(rc, "vdn_hybrid_attn_fwd_profile")
+    return dict(zip(PROFILE_GROUPS, (float(x) for x in ms)))
 
 
 def vdn_vda_scan(shape: Shape, k, v, kt, vt, read_states, text_state, fwd_states, bwd_states,

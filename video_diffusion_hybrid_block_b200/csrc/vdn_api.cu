@@ -219,7 +219,7 @@ bool act_map(CUtensorMap* m, const void* ptr, int64_t rows, const Plan& P, int b
 }
 
 int launch_vda(const Plan& P, const Acts& a, uint8_t* ws, cudaStream_t st, float* text_out,
-               float* fwd_out, float* bwd_out) {
+               float* fwd_out, float* bwd_out, cudaEvent_t after_gram = nullptr) {
   CUtensorMap tk, tv, tkt, tvt, tw, tct;
   if (!act_map(&tk, a.k, P.N, P, 64, ws + P.o_C) || !act_map(&tv, a.v, P.N, P, 64, ws + P.o_C) ||
       !act_map(&tkt, a.kt, P.T, P, 64, ws + P.o_C) ||
@@ -254,6 +254,7 @@ int launch_vda(const Plan& P, const Acts& a, uint8_t* ws, cudaStream_t st, float
   gp.Wmat = reinterpret_cast<float*>(ws + P.o_W);
   k_vda_gram_inv<<<dim3(1 + n_fwd + n_bwd, P.H), kGramThreads, kGramSmemBytes, st>>>(tk, tv, tkt,
                                                                                    tvt, gp);
+  if (after_gram != nullptr) cudaEventRecord(after_gram, st);
   ScanParams sp;
   sp.F = P.F;
   sp.H = P.H;
@@ -397,6 +398,31 @@ int check_ptrs(std::initializer_list<const void*> must, std::initializer_list<co
   return VDN_OK;
 }
 
+// The layer's launches in order: staging (fp32 narrowing / d padding, when
+// needed), Gram + inverse, scans, read-state packing, softmax kernel with the
+// merge epilogue. With `ev` set, ev[0..kProfileGroups] are recorded on the
+// stream at the boundaries of those five groups.
+constexpr int kProfileGroups = 5;
+
+int layer_launches(const Plan& P, const void* q, const void* k, const void* v, const void* kt,
+                   const void* vt, const void* g_s, const void* g_l, const float* rms_w,
+                   void* out, uint8_t* ws, cudaStream_t st, cudaEvent_t* ev) {
+  if (ev != nullptr) cudaEventRecord(ev[0], st);
+  const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, true, true);
+  if (ev != nullptr) cudaEventRecord(ev[1], st);
+  int rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr, ev != nullptr ? ev[2] : nullptr);
+  if (rc != VDN_OK) return rc;
+  if (ev != nullptr) cudaEventRecord(ev[3], st);
+  const float* R = reinterpret_cast<const float*>(ws + P.o_R);
+  k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
+                                                 ws + P.o_Rimg);
+  if (ev != nullptr) cudaEventRecord(ev[4], st);
+  MergeArgs m{g_s, g_l, rms_w, out};
+  rc = launch_bsa(P, a, ws, nullptr, 0, kDPad, nullptr, st, &m);
+  if (ev != nullptr) cudaEventRecord(ev[5], st);
+  return rc;
+}
+
 }  // namespace
 
 extern "C" {
@@ -419,18 +445,50 @@ int vdn_hybrid_attn_fwd(const vdn_shape_t* shape, const void* q, const void* k, 
   if (rc != VDN_OK) return rc;
   rc = common_checks(P, workspace, ws_bytes);
   if (rc != VDN_OK) return rc;
+  return finish(layer_launches(P, q, k, v, kt, vt, g_s, g_l, rms_w, out,
+                               static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream),
+                               nullptr));
+}
+
+int vdn_hybrid_attn_fwd_profile(const vdn_shape_t* shape, const void* q, const void* k,
+                                const void* v, const void* kt, const void* vt, const void* g_s,
+                                const void* g_l, const float* rms_w, void* out, void* workspace,
+                                size_t ws_bytes, void* stream, int iters, float* kernel_ms) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (iters < 1 || iters > 256 || kernel_ms == nullptr) return VDN_ERR_INVALID_ARG;
+  for (int i = 0; i < kProfileGroups; ++i) kernel_ms[i] = 0.f;
+  if (P.N == 0) return VDN_OK;
+  rc = check_ptrs({q, k, v, g_s, g_l, rms_w, out}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, true, true);
-  rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr);
-  if (rc == VDN_OK) {
-    const float* R = reinterpret_cast<const float*>(ws + P.o_R);
-    k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
-                                                   ws + P.o_Rimg);
-    MergeArgs m{g_s, g_l, rms_w, out};
-    rc = launch_bsa(P, a, ws, nullptr, 0, kDPad, nullptr, st, &m);
+  const int ne = (kProfileGroups + 1) * iters;
+  cudaEvent_t* ev = new cudaEvent_t[ne];
+  int made = 0;
+  for (; made < ne; ++made)
+    if (cudaEventCreate(&ev[made]) != cudaSuccess) break;
+  if (made == ne) {
+    for (int it = 0; it < iters && rc == VDN_OK; ++it)
+      rc = layer_launches(P, q, k, v, kt, vt, g_s, g_l, rms_w, out,
+                          static_cast<uint8_t*>(workspace), st, ev + it * (kProfileGroups + 1));
+    rc = finish(rc);
+    if (rc == VDN_OK && cudaStreamSynchronize(st) != cudaSuccess) rc = VDN_ERR_CUDA;
+    for (int it = 0; it < iters && rc == VDN_OK; ++it)
+      for (int g = 0; g < kProfileGroups; ++g) {
+        float ms = 0.f;
+        cudaEvent_t* e = ev + it * (kProfileGroups + 1);
+        if (cudaEventElapsedTime(&ms, e[g], e[g + 1]) != cudaSuccess) rc = VDN_ERR_CUDA;
+        kernel_ms[g] += ms / (float)iters;
+      }
+  } else {
+    rc = VDN_ERR_CUDA;
   }
-  return finish(rc);
+  for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+  delete[] ev;
+  return rc;
 }
 
 int vdn_vda_scan(const vdn_shape_t* shape, const void* k, const void* v, const void* kt,
