@@ -39,7 +39,8 @@ HEADLINE = "hi-res"
 WORKLOADS = ["tiny", "pages-scale", "long-clip", "hi-res", "vda-stress"]
 L2_BYTES = 126 * 2 ** 20
 REF_ROWS = 2048          # query rows per reference-arm step (one head)
-CPU_BASELINE_HEADS = 12  # reference-arm steps in the GPU line's cpu_baseline
+CPU_BASELINE_HEADS = 24  # reference-arm steps in the GPU line's cpu_baseline
+REST_S = 1.0             # idle time before each measurement (power back to idle)
 
 
 # --------------------------------------------------------------- work model --
@@ -308,8 +309,11 @@ def time_launches(torch, stream, fn, n: int, flush=None) -> float:
 
 
 def workload_report(V, torch, w: Workload, stream, steps: int, warmup: int, peaks: dict,
-                    flush_buf) -> dict:
-    """ms/layer, TFLOP/s and per-kernel roofline fractions of one workload."""
+                    flush_buf, gpu_index: int, layer_ms=None) -> dict:
+    """ms/layer, TFLOP/s and per-kernel roofline fractions of one workload.
+    Each measurement starts after REST_S of idle so that none of them runs on
+    clocks lowered by the previous one's power draw; the SM clock sampled
+    over the whole report is recorded beside it."""
     for _ in range(warmup):
         w.layer(V, stream)
     torch.cuda.synchronize()
@@ -317,11 +321,19 @@ def workload_report(V, torch, w: Workload, stream, steps: int, warmup: int, peak
     if rc != 0:
         raise RuntimeError(f"{w.name}: {V.vdn_error_string(rc)}")
     fb = flush_buf if w.flush else None
-    ms = time_launches(torch, stream, lambda: w.layer(V, stream), steps, fb)
-    kern = V.vdn_hybrid_attn_fwd_profile(w.shape, w.dev["q"], w.dev["k"], w.dev["v"],
-                                         w.dev["kt"], w.dev["vt"], w.dev["g_s"], w.dev["g_l"],
-                                         w.rms_w, w.out, w.ws, iters=min(steps, 20),
-                                         stream=stream)
+    with ClockSampler(gpu_index) as clk:
+        if layer_ms is None:
+            time.sleep(REST_S)
+            layer_ms = time_launches(torch, stream, lambda: w.layer(V, stream), steps, fb)
+        time.sleep(REST_S)
+        kern = V.vdn_hybrid_attn_fwd_profile(w.shape, w.dev["q"], w.dev["k"], w.dev["v"],
+                                             w.dev["kt"], w.dev["vt"], w.dev["g_s"], w.dev["g_l"],
+                                             w.rms_w, w.out, w.ws, iters=min(steps, 10),
+                                             stream=stream)
+        extra = {}
+        if w.inp["d"] == 128 and w.inp["dtype"] == "bf16":
+            extra = standalone_kernels(V, torch, w, stream, steps)
+    ms = layer_ms
     fl = w.fl
     merged_flop = fl["softmax"] + fl["readout"]
     t_sm = kern["softmax_merge"]
@@ -337,33 +349,14 @@ def workload_report(V, torch, w: Workload, stream, steps: int, warmup: int, peak
             "frac_sustained": round(merged_flop / (t_sm * 1e-3) / 1e12 / peaks["bf16_sustained"], 4),
         },
     }
-    if w.inp["d"] == 128 and w.inp["dtype"] == "bf16":
-        # softmax branch alone (no merge epilogue), and the standalone merge
-        o_soft = torch.empty(w.dev["q"].shape, dtype=torch.bfloat16, device="cuda")
-        nb = w.shape.nb
-        R = torch.empty((nb, w.inp["H"], 128, 128), device="cuda")
-        d = w.dev
-        V.vdn_vda_scan(w.shape, d["k"], d["v"], d["kt"], d["vt"], R, None, None, None, w.ws,
-                       stream)
-
-        def bsa():
-            V.vdn_bsa_fwd(w.shape, d["q"], d["k"], d["v"], d["kt"], d["vt"], o_soft, None, w.ws,
-                          stream)
-
-        def merge():
-            V.vdn_gate_merge(w.shape, d["q"], R, o_soft, d["g_s"], d["g_l"], w.rms_w, w.out, w.ws,
-                             stream)
-
-        bsa()
-        t_bsa = time_launches(torch, stream, bsa, max(3, steps // 2))
-        merge()
-        t_merge = time_launches(torch, stream, merge, max(5, steps))
+    if extra:
+        t_bsa = extra["bsa_ms"]
         rep["softmax_only"] = {"kernel": "k_bsa_fwd", "ms": round(t_bsa, 4),
                                "frac_burst": round(fl["softmax"] / (t_bsa * 1e-3) / 1e12
                                                    / peaks["bf16_tflops"], 4)}
         hbm = {}
         for key, t in (("gram_inv", kern["gram_inv"]), ("scan", kern["scan"]),
-                       ("pack", kern["pack"]), ("gate_merge", t_merge)):
+                       ("pack", kern["pack"]), ("gate_merge", extra["merge_ms"])):
             b = w.bytes[key]
             gbs = b / (t * 1e-3) / 1e9 if t > 0 else None
             hbm[key] = {"bytes": int(b), "ms": round(t, 4),
@@ -371,13 +364,39 @@ def workload_report(V, torch, w: Workload, stream, steps: int, warmup: int, peak
                         "frac": round(gbs / peaks["hbm_gbs"], 4) if gbs else None}
         hbm["gate_merge"]["kernel"] = "k_readout_merge_tma (vdn_gate_merge)"
         rep["hbm"] = hbm
-        del o_soft, R
-    # outputs are still valid after the helper runs (same computation)
+    c = clk.summary()
+    rep["sm_mhz"] = c["sm_mhz"]
+    rep["clock_reasons"] = c["reasons"]
     torch.cuda.synchronize()
     rc = V.vdn_get_device_error()
     if rc != 0:
         raise RuntimeError(f"{w.name}: {V.vdn_error_string(rc)}")
     return rep
+
+
+def standalone_kernels(V, torch, w: Workload, stream, steps: int) -> dict:
+    """The softmax branch alone (no merge epilogue) and the standalone
+    readout + merge kernel, each timed by itself after a rest."""
+    o_soft = torch.empty(w.dev["q"].shape, dtype=torch.bfloat16, device="cuda")
+    R = torch.empty((w.shape.nb, w.inp["H"], 128, 128), device="cuda")
+    d = w.dev
+    V.vdn_vda_scan(w.shape, d["k"], d["v"], d["kt"], d["vt"], R, None, None, None, w.ws, stream)
+
+    def bsa():
+        V.vdn_bsa_fwd(w.shape, d["q"], d["k"], d["v"], d["kt"], d["vt"], o_soft, None, w.ws,
+                      stream)
+
+    def merge():
+        V.vdn_gate_merge(w.shape, d["q"], R, o_soft, d["g_s"], d["g_l"], w.rms_w, w.out, w.ws,
+                         stream)
+
+    bsa()
+    time.sleep(REST_S)
+    t_bsa = time_launches(torch, stream, bsa, max(3, steps // 2))
+    merge()
+    time.sleep(REST_S)
+    t_merge = time_launches(torch, stream, merge, max(5, steps))
+    return dict(bsa_ms=t_bsa, merge_ms=t_merge)
 
 
 def run_cuda(args) -> None:
@@ -411,6 +430,7 @@ def run_cuda(args) -> None:
         raise RuntimeError(V.vdn_error_string(rc))
     flush_buf = torch.empty(64 * 2 ** 20, dtype=torch.float32, device="cuda")  # 256 MiB
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    time.sleep(REST_S)
     with ClockSampler(local) as clk:
         if w.flush:
             barrier()
@@ -476,13 +496,14 @@ def run_cuda(args) -> None:
     e2e_ms = max_over_ranks(dist, g0.elapsed_time(g1) / args.steps, "cuda")
     del sets[1], outs[1]
 
-    # ---- every workload (the headline's object is measured on its buffers)
+    # ---- every workload; the headline's report reuses its layer time
     reports = {}
     names = [args.workload] if args.workloads == "none" else WORKLOADS
     for name in names:
         ww = w if name == args.workload else Workload(name, V, torch)
         reports[name] = workload_report(V, torch, ww, stream, args.steps, args.warmup, peaks,
-                                        flush_buf)
+                                        flush_buf, local,
+                                        layer_ms=ms if name == args.workload else None)
         if ww is not w:
             del ww
             torch.cuda.empty_cache()
