@@ -84,6 +84,10 @@ extern "C" {
 
 typedef enum { VDN_BF16 = 0, VDN_F32 = 1 } vdn_dtype_t;
 
+/* Arithmetic of the per-branch output projections. */
+#define VDN_PROJ_BF16 0 /* bf16 operands, fp32 accumulation                  */
+#define VDN_PROJ_FP8 1  /* e4m3 operands with per-row scales, fp32 accumulation */
+
 typedef struct vdn_shape {
   int32_t F;            /* latent frames                                   */
   int32_t T;            /* text tokens (0 allowed: S_text = 0)             */
@@ -108,6 +112,61 @@ int vdn_hybrid_attn_fwd(const vdn_shape_t* shape, const void* q, const void* k,
                         const void* v, const void* kt, const void* vt,
                         const void* g_s, const void* g_l, const float* rms_w,
                         void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Per-branch output projections. Each branch has its own sigmoid gate and its
+ * own output projection before the merge [nav.superapi.store page, Technical
+ * Principles, Gated Fusion Mechanism; openi.cn page, 技术原理, last
+ * paragraph]; the pages run these linears in FP8. Reading implemented (gates
+ * are per token and head, so they act before the projection):
+ *   a_s = sigmoid(g_s) o_soft,  a_l = sigmoid(g_l) RMSNorm(o_lin)   [N, H, d]
+ *   y   = W_s a_s + W_l a_l = [a_s | a_l] w_o^T,  w_o = [W_s | W_l] [D, 2 H d]
+ * (heads flattened as h * d + j; w_o = [I | I] gives vdn_hybrid_attn_fwd's
+ * output). These entry points need bf16 activations with d = 128
+ * (VDN_ERR_UNSUPPORTED otherwise).
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes of vdn_hybrid_attn_proj_fwd (0 if the arguments are
+ * invalid): the layer's workspace plus the gated branches [N, 2H, 128] bf16
+ * and, for VDN_PROJ_FP8, their e4m3 codes [N, 2H, 128] and row scales [N]. */
+size_t vdn_proj_workspace_bytes(const vdn_shape_t* shape, int D, int precision);
+
+/* The layer up to the merge, with the two gated branches kept apart:
+ * branches [N, 2H, d] bf16 gets a_s in heads 0..H-1 and a_l in heads
+ * H..2H-1 (so row n is the [2 H d] input of the projection). */
+int vdn_hybrid_attn_branches(const vdn_shape_t* shape, const void* q, const void* k,
+                             const void* v, const void* kt, const void* vt,
+                             const void* g_s, const void* g_l, const float* rms_w,
+                             void* branches, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* y [M, D] bf16 = a [M, K] w [D, K]^T, fp32 accumulation (row-major, K
+ * contiguous in both operands; w is laid out like a linear layer's weight).
+ * VDN_PROJ_BF16: a, w bf16, scales ignored (may be NULL).
+ * VDN_PROJ_FP8: a, w e4m3 codes (1 byte each), y[m, n] = a_scale[m] *
+ * w_scale[n] * sum_k a[m, k] w[n, k]; a_scale [M], w_scale [D] fp32.
+ * K % 16 == 0, K >= 16, D % 8 == 0, D >= 8, M >= 0. */
+int vdn_linear(const void* a, const float* a_scale, const void* w, const float* w_scale,
+               int64_t M, int K, int D, int precision, void* y, void* stream);
+
+/* Per-row e4m3 quantisation of x [rows, K] bf16 (K % 16 == 0):
+ * scales[r] = amax_r / 448 (1 for an all-zero row) and codes[r, k] =
+ * e4m3(x[r, k] * (448 / amax_r)) rounded to nearest even with saturation,
+ * all in fp32. Used for the weights (once, per output channel) and, inside
+ * vdn_hybrid_attn_proj_fwd, for the gated branches (per token). */
+int vdn_quantize_rows_e4m3(const void* x, int64_t rows, int K, void* codes, float* scales,
+                           void* stream);
+
+/* Whole layer with the per-branch output projections: y [N, D] bf16.
+ * VDN_PROJ_BF16: w_o [D, 2 H d] bf16, w_scale NULL. VDN_PROJ_FP8: w_o holds
+ * e4m3 codes [D, 2 H d] and w_scale [D] as written by vdn_quantize_rows_e4m3;
+ * the gated branches are quantised per token on the fly. workspace must hold
+ * vdn_proj_workspace_bytes(shape, D, precision). */
+int vdn_hybrid_attn_proj_fwd(const vdn_shape_t* shape, const void* q, const void* k,
+                             const void* v, const void* kt, const void* vt,
+                             const void* g_s, const void* g_l, const float* rms_w,
+                             const void* w_o, const float* w_scale, int D, int precision,
+                             void* y, void* workspace, size_t ws_bytes, void* stream);
 
 /* Measurement helper (no paper counterpart). Runs vdn_hybrid_attn_fwd (same
  * arguments) `iters` times (1..256) on `stream` with CUDA events recorded on

@@ -39,11 +39,16 @@ library implements too):
   [w0, w1] is b's window of frames and S_fwd[0] = S_bwd[F-1] = S_text;
 * o_lin = q^T R_b (q not normalised); RMSNorm over d per head, eps 1e-6,
   weight w[h, :];
-* out = sigmoid(g_s) o_soft + sigmoid(g_l) RMSNorm(o_lin).
+* out = sigmoid(g_s) o_soft + sigmoid(g_l) RMSNorm(o_lin);
+* with per-branch output projections (w_o = [W_s | W_l], [D, 2 H d]):
+  y = W_s (sigmoid(g_s) o_soft) + W_l (sigmoid(g_l) RMSNorm(o_lin)), heads
+  flattened as h * d + j.
 
 Parity is pinned by tests/test_oracle_pins.py (dense-mask equivalence,
 Sherman-Morrison, ridge closed form, orthonormal-key delta steps, fixed point,
-non-expansiveness, pair-set coverage, RMSNorm closed form). The comparison of
+non-expansiveness, pair-set coverage, RMSNorm closed form, readout
+orientation, text start of both scans) and tests/test_oracle_proj.py
+(projection: identity weights, brute-force loops, gate limits). The comparison of
 the pair split with the pages' ~52%/48% and +3.57% figures is reported, not
 pinned ("parity unpinned" for those two statistics: no uniform frame layout
 reproduces both figures).
@@ -307,3 +312,51 @@ def layer(inp: dict) -> dict:
         R=np.stack([r["states"]["R"] for r in res], axis=1),
         states=[r["states"] for r in res],
     )
+
+
+# ---------------------------------------------------------------------------
+# Per-branch output projections
+# ---------------------------------------------------------------------------
+#
+# Each branch carries its own content-dependent sigmoid gate and its own
+# output projection, and the projected branches are merged by a sum
+# [nav.superapi.store page, Technical Principles, "Gated Fusion Mechanism";
+# openi.cn page, "技术原理：局部精确、远程压缩", last paragraph]. With the gate
+# logits given per token and per head, the gate is applied per head before
+# the projection:
+#   y = W_s (sigmoid(g_s) o_soft) + W_l (sigmoid(g_l) RMSNorm(o_lin))
+# where o_soft, o_lin are flattened over heads (index h * d + j). Written as
+# one matrix: y = w_o @ [a_s ; a_l], w_o = [W_s | W_l] of shape [D, 2 H d].
+# With W_s = W_l = I (D = H d) this is the merged layer output above.
+
+
+def gated_branches_head(inp: dict, h: int, rows=None) -> dict:
+    """The two gated branch outputs of one head, before any projection:
+    a_s = sigmoid(g_s) o_soft, a_l = sigmoid(g_l) RMSNorm(o_lin)."""
+    res = layer_head(inp, h, rows=rows)
+    N = int(np.asarray(inp["off"])[-1])
+    all_rows = np.arange(N) if rows is None else np.asarray(rows)
+    a_s = sigmoid(inp["g_s"][all_rows, h])[:, None] * res["o_soft"]
+    a_l = sigmoid(inp["g_l"][all_rows, h])[:, None] * rmsnorm(res["o_lin"], inp["rms_w"][h],
+                                                               inp["eps"])
+    return dict(a_s=a_s, a_l=a_l, out=res["out"])
+
+
+def gated_branches(inp: dict, rows=None) -> np.ndarray:
+    """[rows, 2, H, d]: branch 0 = a_s, branch 1 = a_l, every head."""
+    H = inp["H"]
+    parts = [gated_branches_head(inp, h, rows) for h in range(H)]
+    a_s = np.stack([p["a_s"] for p in parts], axis=1)
+    a_l = np.stack([p["a_l"] for p in parts], axis=1)
+    return np.stack([a_s, a_l], axis=1)
+
+
+def output_projection(branches, w_o) -> np.ndarray:
+    """y = [a_s ; a_l] projected by w_o [D, 2 H d]: branches [rows, 2, H, d]."""
+    b = np.asarray(branches, np.float64)
+    return b.reshape(b.shape[0], -1) @ np.asarray(w_o, np.float64).T
+
+
+def layer_proj(inp: dict, w_o, rows=None) -> np.ndarray:
+    """The layer with per-branch output projections: [rows, D]."""
+    return output_projection(gated_branches(inp, rows), w_o)

@@ -187,3 +187,55 @@ def test_binding_rejects_tensors_the_kernels_would_overrun():
                        ws_bytes=1 << 40)
     with pytest.raises(ValueError, match="soft_pairs"):
         V.vdn_pair_audit(sh, t(10 * 10, torch.int64), FAKE)
+
+
+# ------------------------------------------------ per-branch projections ---
+
+def test_proj_workspace_bytes(lib):
+    s = shape(H=3)
+    N = int(s.N)
+    base = V.vdn_workspace_bytes(s)
+    K = 2 * 3 * 128
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert V.vdn_proj_workspace_bytes(s, 384, B.VDN_PROJ_BF16) == base + al(N * K * 2)
+    assert V.vdn_proj_workspace_bytes(s, 384, B.VDN_PROJ_FP8) == \
+        base + al(N * K * 2) + al(N * K) + al(N * 4)
+    # bf16 with d = 128 only; D a positive multiple of 8; known precision
+    assert V.vdn_proj_workspace_bytes(shape(d=64), 384, 0) == 0
+    assert V.vdn_proj_workspace_bytes(shape(dtype=1), 384, 0) == 0
+    assert V.vdn_proj_workspace_bytes(s, 12, 0) == 0
+    assert V.vdn_proj_workspace_bytes(s, 384, 2) == 0
+
+
+@pytest.mark.parametrize("M,K,D,prec,code", [
+    (-1, 64, 64, 0, B.VDN_ERR_INVALID_ARG), (10, 8, 64, 0, B.VDN_ERR_INVALID_ARG),
+    (10, 72, 64, 0, B.VDN_ERR_INVALID_ARG), (10, 64, 4, 0, B.VDN_ERR_INVALID_ARG),
+    (10, 64, 68, 0, B.VDN_ERR_INVALID_ARG), (10, 64, 64, 3, B.VDN_ERR_UNSUPPORTED)])
+def test_linear_rejects_bad_sizes(lib, M, K, D, prec, code):
+    assert lib.vdn_linear(FAKE, FAKE, FAKE, FAKE, M, K, D, prec, FAKE, 0) == code
+
+
+def test_linear_and_quant_pointer_checks(lib):
+    assert lib.vdn_linear(None, None, FAKE, None, 10, 64, 64, 0, FAKE, 0) == B.VDN_ERR_INVALID_ARG
+    assert lib.vdn_linear(FAKE_MIS, None, FAKE, None, 10, 64, 64, 0, FAKE, 0) == B.VDN_ERR_MISALIGNED
+    # e4m3 needs both scale vectors
+    assert lib.vdn_linear(FAKE, None, FAKE, FAKE, 10, 64, 64, 1, FAKE, 0) == B.VDN_ERR_INVALID_ARG
+    assert lib.vdn_linear(FAKE, FAKE, FAKE, FAKE_MIS, 10, 64, 64, 1, FAKE, 0) == B.VDN_ERR_MISALIGNED
+    assert lib.vdn_quantize_rows_e4m3(FAKE, 10, 24, FAKE, FAKE, 0) == B.VDN_ERR_INVALID_ARG
+    assert lib.vdn_quantize_rows_e4m3(None, 10, 32, FAKE, FAKE, 0) == B.VDN_ERR_INVALID_ARG
+    assert lib.vdn_quantize_rows_e4m3(FAKE, 10, 32, FAKE_MIS, FAKE, 0) == B.VDN_ERR_MISALIGNED
+    assert lib.vdn_quantize_rows_e4m3(FAKE, 0, 32, None, None, 0) == B.VDN_OK
+
+
+def test_proj_layer_checks(lib):
+    s = shape()
+    need = V.vdn_proj_workspace_bytes(s, 256, 1)
+    args = [FAKE] * 8
+    assert lib.vdn_hybrid_attn_proj_fwd(s.ref, *args, FAKE, None, 256, 1, FAKE, FAKE, need, 0) == \
+        B.VDN_ERR_INVALID_ARG
+    assert lib.vdn_hybrid_attn_proj_fwd(s.ref, *args, FAKE, FAKE, 256, 1, FAKE, FAKE, need - 1,
+                                        0) == B.VDN_ERR_WORKSPACE_TOO_SMALL
+    assert lib.vdn_hybrid_attn_proj_fwd(shape(d=64).ref, *args, FAKE, FAKE, 256, 1, FAKE, FAKE,
+                                        need, 0) == B.VDN_ERR_UNSUPPORTED
+    assert lib.vdn_hybrid_attn_branches(shape(dtype=1).ref, *([FAKE] * 9), FAKE, need, 0) == \
+        B.VDN_ERR_UNSUPPORTED

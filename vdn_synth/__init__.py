@@ -21,6 +21,8 @@ q, k, v, kt, vt, g_s, g_l.
 * gate logits g_s, g_l ~ N(0, 1) with shape [N, H]; RMSNorm weight = 1 [H, d].
 * bf16 workloads round every float input to bf16 (round to nearest even);
   the returned float32 arrays then hold exactly the bf16 values.
+* output-projection weights (make_proj_weight): w_o [D, 2 H d] ~
+  N(0, 1) / sqrt(2 H d), default_rng(seed + 1000), bf16.
 """
 from __future__ import annotations
 
@@ -123,6 +125,16 @@ def make_inputs_from(F, sizes, T, H, d, dtype="bf16", seed=0, k_lowrank=None,
                H=H, d=d, N=N, dtype=dtype, block_frames=BLOCK_FRAMES,
                lam=LAMBDA, eps=RMS_EPS)
     return out
+
+
+def make_proj_weight(H: int, d: int, D: int | None = None, seed: int = 0) -> np.ndarray:
+    """Synthetic output-projection weight w_o [D, 2 H d] (D = H d by default):
+    N(0, 1) / sqrt(2 H d) float32 from default_rng(seed + 1000), rounded to
+    bf16. There are no trained weights; this only sets shapes and scale."""
+    D = H * d if D is None else D
+    rng = np.random.default_rng(seed + 1000)
+    w = rng.standard_normal((D, 2 * H * d), dtype=np.float32) / np.float32(np.sqrt(2 * H * d))
+    return bf16_round(w)
 
 
 def make_inputs(name: str, seed: int = 0) -> dict:

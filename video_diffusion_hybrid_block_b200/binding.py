@@ -25,6 +25,9 @@ VDN_ERR_DEVICE = -7
 VDN_BF16 = 0
 VDN_F32 = 1
 
+VDN_PROJ_BF16 = 0
+VDN_PROJ_FP8 = 1
+
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdn.so")
 
 
@@ -57,6 +60,14 @@ _SIGS = {
     "vdn_hybrid_attn_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 9 + [_P, _SZ, _P]),
     "vdn_hybrid_attn_fwd_profile": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 9
                                     + [_P, _SZ, _P, ctypes.c_int, ctypes.POINTER(ctypes.c_float)]),
+    "vdn_proj_workspace_bytes": (_SZ, [ctypes.POINTER(vdn_shape_t), ctypes.c_int, ctypes.c_int]),
+    "vdn_hybrid_attn_branches": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 9
+                                 + [_P, _SZ, _P]),
+    "vdn_linear": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int, _P, _P]),
+    "vdn_quantize_rows_e4m3": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int, _P, _P, _P]),
+    "vdn_hybrid_attn_proj_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 8
+                                 + [_P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _SZ, _P]),
     "vdn_vda_scan": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 8 + [_P, _SZ, _P]),
     "vdn_gate_merge": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
     "vdn_bsa_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
@@ -285,6 +296,78 @@ def vdn_selftest_wait_timeout(limit_ns: int, tmem_cols: int = 0, stream=None):
 
 def vdn_get_device_error() -> int:
     return int(load_library().vdn_get_device_error())
+
+
+# ------------------------------------------------ per-branch projections ---
+
+def _proj_K(shape: Shape) -> int:
+    return 2 * shape.H * shape.d
+
+
+def vdn_proj_workspace_bytes(shape: Shape, D: int, precision: int) -> int:
+    return int(load_library().vdn_proj_workspace_bytes(shape.ref, int(D), int(precision)))
+
+
+def alloc_proj_workspace(shape: Shape, D: int, precision: int, device=None) -> torch.Tensor:
+    n = vdn_proj_workspace_bytes(shape, D, precision)
+    if n == 0:
+        raise VdnError(VDN_ERR_INVALID_ARG, "vdn_proj_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def vdn_hybrid_attn_branches(shape: Shape, q, k, v, kt, vt, g_s, g_l, rms_w, branches, workspace,
+                             stream=None, ws_bytes=None):
+    _check_acts(shape, q, k, v, kt, vt, g_s, g_l)
+    _need(rms_w, shape.H * shape.d, 4, "rms_w")
+    _need(branches, shape.N * _proj_K(shape), 2, "branches")
+    rc = load_library().vdn_hybrid_attn_branches(
+        shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(g_s), _ptr(g_l),
+        _ptr(rms_w), _ptr(branches), _ptr(workspace), _nbytes(workspace, ws_bytes),
+        _stream(stream))
+    _check(rc, "vdn_hybrid_attn_branches")
+    return branches
+
+
+def vdn_linear(a, a_scale, w, w_scale, M: int, K: int, D: int, precision: int, y, stream=None):
+    """y [M, D] bf16 = a [M, K] w [D, K]^T (e4m3 codes with row scales for
+    VDN_PROJ_FP8)."""
+    es = 1 if precision == VDN_PROJ_FP8 else 2
+    _need(a, M * K, es, "a")
+    _need(w, D * K, es, "w")
+    _need(y, M * D, 2, "y")
+    if precision == VDN_PROJ_FP8:
+        _need(a_scale, M, 4, "a_scale")
+        _need(w_scale, D, 4, "w_scale")
+    rc = load_library().vdn_linear(_ptr(a), _ptr(a_scale), _ptr(w), _ptr(w_scale), int(M), int(K),
+                                   int(D), int(precision), _ptr(y), _stream(stream))
+    _check(rc, "vdn_linear")
+    return y
+
+
+def vdn_quantize_rows_e4m3(x, rows: int, K: int, codes, scales, stream=None):
+    _need(x, rows * K, 2, "x")
+    _need(codes, rows * K, 1, "codes")
+    _need(scales, rows, 4, "scales")
+    rc = load_library().vdn_quantize_rows_e4m3(_ptr(x), int(rows), int(K), _ptr(codes),
+                                               _ptr(scales), _stream(stream))
+    _check(rc, "vdn_quantize_rows_e4m3")
+    return codes, scales
+
+
+def vdn_hybrid_attn_proj_fwd(shape: Shape, q, k, v, kt, vt, g_s, g_l, rms_w, w_o, w_scale, D: int,
+                             precision: int, y, workspace, stream=None, ws_bytes=None):
+    _check_acts(shape, q, k, v, kt, vt, g_s, g_l)
+    _need(rms_w, shape.H * shape.d, 4, "rms_w")
+    _need(w_o, D * _proj_K(shape), 1 if precision == VDN_PROJ_FP8 else 2, "w_o")
+    if precision == VDN_PROJ_FP8:
+        _need(w_scale, D, 4, "w_scale")
+    _need(y, shape.N * D, 2, "y")
+    rc = load_library().vdn_hybrid_attn_proj_fwd(
+        shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(g_s), _ptr(g_l),
+        _ptr(rms_w), _ptr(w_o), _ptr(w_scale), int(D), int(precision), _ptr(y), _ptr(workspace),
+        _nbytes(workspace, ws_bytes), _stream(stream))
+    _check(rc, "vdn_hybrid_attn_proj_fwd")
+    return y
 
 
 def alloc_workspace(shape: Shape, device=None) -> torch.Tensor:

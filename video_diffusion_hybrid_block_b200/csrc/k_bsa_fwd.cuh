@@ -90,12 +90,17 @@ struct BsaParams {
   int tma_out;           // out is bf16 [N][H][128]: full tiles leave through a TMA store
 };
 
-template <bool kMerge>
+// kMode: 0 = softmax branch only (o_soft, lse); 1 = merged layer output;
+// 2 = the two gated branches written side by side for the per-branch output
+// projections (out is [N][2H][128] bf16: head h holds sigmoid(g_s) O / l,
+// head H + h holds sigmoid(g_l) w * o_lin / rms).
+template <int kMode>
 __global__ void __launch_bounds__(kBsaThreads, 1)
     k_bsa_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkt,
               const __grid_constant__ CUtensorMap tvt, const __grid_constant__ CUtensorMap tout,
               const BsaParams p) {
+  constexpr bool kMerge = kMode != 0;
   const int pair = blockIdx.x, h = blockIdx.y;
   const int b = block_in_visit_order(blockIdx.z, num_blocks(p.F, p.bf));
   int q0, q1;
@@ -429,6 +434,50 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       // buffer and one TMA store; otherwise each thread stores its row
       const bool via_tma = p.tma_out && (qs + tile * kTile + kTile <= q1);
       const uint32_t stage = sQ + (uint32_t)tile * 32768u;
+      if constexpr (kMode == 2) {
+        // pass 0: soft branch into head h, pass 1: linear branch into head H + h
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t x[32];
+            tmem_ld32((pass == 0 ? tO : tS) + (uint32_t)(c * 32), x);
+            tmem_ld_wait(x);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int c0 = c * 32 + u * 8;
+              float y[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                y[e] = pass == 0 ? a_s * __uint_as_float(x[u * 8 + e])
+                                 : a_l * w_sm[c0 + e] * __uint_as_float(x[u * 8 + e]);
+              const uint32_t w0 = pack_bf16x2(y[0], y[1]), w1 = pack_bf16x2(y[2], y[3]);
+              const uint32_t w2 = pack_bf16x2(y[4], y[5]), w3 = pack_bf16x2(y[6], y[7]);
+              if (via_tma) {
+                st_shared_v4(stage + (uint32_t)(c0 >> 6) * 16384u +
+                                 sw128_off((uint32_t)r, (uint32_t)((c0 & 63) >> 3)),
+                             w0, w1, w2, w3);
+              } else if (store) {
+                const int64_t ob = ((int64_t)row * 2 * p.H + pass * p.H + h) * kDPad + c0;
+                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + ob) =
+                    make_uint4(w0, w1, w2, w3);
+              }
+            }
+          }
+          if (via_tma) {
+            fence_proxy_async_smem();
+            named_barrier_sync(2 + tile, 128);
+            if (r == 0 && ok) {
+              const int row0 = qs + tile * kTile;
+              tma_store_3d(&tout, stage, 0, pass * p.H + h, row0);
+              tma_store_3d(&tout, stage + 16384u, 64, pass * p.H + h, row0);
+              bulk_commit_group();
+              bulk_wait_all();  // the staging buffer is refilled by the next pass
+            }
+            named_barrier_sync(2 + tile, 128);
+          }
+        }
+      } else {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32], z[32];
@@ -470,6 +519,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
           bulk_commit_group();
           bulk_wait_all();
         }
+      }
       }
     }
   }

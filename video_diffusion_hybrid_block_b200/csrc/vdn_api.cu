@@ -12,6 +12,7 @@
 #include "../../include/vdn.h"
 #include "k_audit.cuh"
 #include "k_bsa_fwd.cuh"
+#include "k_linear.cuh"
 #include "k_merge.cuh"
 #include "k_prepare.cuh"
 #include "k_vda.cuh"
@@ -66,6 +67,23 @@ bool map_mat(CUtensorMap* m, const void* ptr, int64_t rows, int box_rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+// [rows, inner] row-major matrix of 2-byte (bf16) or 1-byte (raw e4m3)
+// elements; box {box_inner, box_rows}, 128-byte swizzle (box_inner x element
+// size must be 128 B).
+bool map_rows(CUtensorMap* m, const void* ptr, int64_t inner, int64_t rows, int esize,
+              int box_inner, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(inner * esize)};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+             const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 __global__ void k_sum_states(const float* a, const float* b, float* out, int64_t n, int d) {
   // out[(bh, i, j)] = a[(bh, i, j)] + b[(bh, i, j)] with a, b padded to 128 x 128
@@ -149,10 +167,16 @@ bool set_smem_attrs() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (done[dev]) return true;
-  bool ok = cudaFuncSetAttribute(k_bsa_fwd<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  bool ok = cudaFuncSetAttribute(k_bsa_fwd<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kBsaSmemBytes) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(k_bsa_fwd<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  ok = ok && cudaFuncSetAttribute(k_bsa_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBsaMergeSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_bsa_fwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kBsaMergeSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_linear<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kLinSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_linear<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kLinSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_vda_gram_inv, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kGramSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_vda_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -277,6 +301,7 @@ struct MergeArgs {
   const void* g_l;
   const float* rms_w;
   void* out;
+  bool branches = false;  // out is [N][2H][128] bf16: the two gated branches
 };
 
 // Softmax branch; with `merge` set, the readout + gated merge run in its
@@ -293,7 +318,11 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
     return VDN_ERR_CUDA;
   // the merged output leaves by TMA stores when it is bf16 with d = 128
   const bool tma_out = merge != nullptr && P.dtype == VDN_BF16 && P.d == kDPad;
-  if (!act_map(&tout, tma_out ? merge->out : a.q, P.N, P, 128, ws + P.o_C)) return VDN_ERR_CUDA;
+  if (merge != nullptr && merge->branches) {
+    if (!map_act(&tout, merge->out, P.N, 2 * P.H, 128)) return VDN_ERR_CUDA;
+  } else if (!act_map(&tout, tma_out ? merge->out : a.q, P.N, P, 128, ws + P.o_C)) {
+    return VDN_ERR_CUDA;
+  }
   BsaParams bp;
   memset(&bp, 0, sizeof(bp));
   bp.off = P.off_dev;
@@ -311,7 +340,7 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
   // blocks on z (dispatched last), visited interior-first by the kernel
   const dim3 grid((P.max_qtiles + 1) / 2, P.H, P.nb);
   if (merge == nullptr) {
-    k_bsa_fwd<false><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
+    k_bsa_fwd<0><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
   } else {
     bp.rimg = ws + P.o_Rimg;
     bp.g_s = merge->g_s;
@@ -322,7 +351,10 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
     bp.out = merge->out;
     bp.out_f32 = (P.dtype == VDN_F32);
     bp.tma_out = tma_out ? 1 : 0;
-    k_bsa_fwd<true><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
+    if (merge->branches)
+      k_bsa_fwd<2><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
+    else
+      k_bsa_fwd<1><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
   }
   return VDN_OK;
 }
@@ -398,6 +430,90 @@ int check_ptrs(std::initializer_list<const void*> must, std::initializer_list<co
   return VDN_OK;
 }
 
+// ---------------------------------------------------------- projections --
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+int check_linear_args(const void* a, const float* a_scale, const void* w, const float* w_scale,
+                      int64_t M, int K, int D, int precision, const void* y) {
+  if (precision != VDN_PROJ_BF16 && precision != VDN_PROJ_FP8) return VDN_ERR_UNSUPPORTED;
+  if (M < 0 || K < 16 || D < 8 || (K % 16) != 0 || (D % 8) != 0) return VDN_ERR_INVALID_ARG;
+  if (M > ((int64_t)1 << 31) - 1 || (int64_t)D * K > ((int64_t)1 << 40)) return VDN_ERR_UNSUPPORTED;
+  for (const void* p : {a, w, y}) {
+    if (p == nullptr) return VDN_ERR_INVALID_ARG;
+    if (!aligned16(p)) return VDN_ERR_MISALIGNED;
+  }
+  if (precision == VDN_PROJ_FP8) {
+    if (a_scale == nullptr || w_scale == nullptr) return VDN_ERR_INVALID_ARG;
+    if (!aligned16(a_scale) || !aligned16(w_scale)) return VDN_ERR_MISALIGNED;
+  }
+  return VDN_OK;
+}
+
+// y [M, D] bf16 = A [M, K] W [D, K]^T (times the row / column scales for e4m3)
+int launch_linear(const void* a, const float* a_scale, const void* w, const float* w_scale,
+                  int64_t M, int K, int D, int precision, void* y, cudaStream_t st) {
+  if (M == 0) return VDN_OK;
+  const bool fp8 = precision == VDN_PROJ_FP8;
+  const int es = fp8 ? 1 : 2;
+  const int bk = fp8 ? 128 : 64;
+  CUtensorMap ta, tw, ty;
+  if (!map_rows(&ta, a, K, M, es, bk, kLinBM) || !map_rows(&tw, w, K, D, es, bk, kLinBN) ||
+      !map_rows(&ty, y, D, M, 2, 64, kLinBM))
+    return VDN_ERR_CUDA;
+  LinParams lp;
+  lp.M = (int)M;
+  lp.K = K;
+  lp.D = D;
+  lp.tiles_m = (int)((M + kLinBM - 1) / kLinBM);
+  lp.tiles_n = (D + kLinBN - 1) / kLinBN;
+  lp.a_scale = a_scale;
+  lp.w_scale = w_scale;
+  const int tiles = lp.tiles_m * lp.tiles_n;
+  const int sms = sm_count();
+  if (sms <= 0) return VDN_ERR_CUDA;
+  const int grid = imin(tiles, sms);
+  if (fp8)
+    k_linear<true><<<grid, kLinThreads, kLinSmemBytes, st>>>(ta, tw, ty, lp);
+  else
+    k_linear<false><<<grid, kLinThreads, kLinSmemBytes, st>>>(ta, tw, ty, lp);
+  return VDN_OK;
+}
+
+void launch_quant(const void* x, int64_t rows, int K, void* codes, float* scales, cudaStream_t st) {
+  if (rows == 0) return;
+  const int warps = 8;
+  k_quant_rows_e4m3<<<(unsigned)((rows + warps - 1) / warps), warps * 32, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, K, static_cast<uint8_t*>(codes), scales);
+}
+
+// Workspace of the projected layer: the layer's own workspace, then the
+// gated branches [N, 2H, 128] bf16 and, for e4m3, their codes and row scales.
+struct ProjPlan {
+  size_t o_branches, o_codes, o_scales, total;
+};
+
+int make_proj_plan(const Plan& P, int D, int precision, ProjPlan* Q) {
+  if (P.dtype != VDN_BF16 || P.d != kDPad) return VDN_ERR_UNSUPPORTED;
+  if (precision != VDN_PROJ_BF16 && precision != VDN_PROJ_FP8) return VDN_ERR_UNSUPPORTED;
+  if (D < 8 || (D % 8) != 0) return VDN_ERR_INVALID_ARG;
+  const size_t K = (size_t)2 * P.H * kDPad;
+  size_t o = P.total;
+  Q->o_branches = o;
+  o += align256((size_t)P.N * K * 2);
+  Q->o_codes = o;
+  o += precision == VDN_PROJ_FP8 ? align256((size_t)P.N * K) : 0;
+  Q->o_scales = o;
+  o += precision == VDN_PROJ_FP8 ? align256((size_t)P.N * 4) : 0;
+  Q->total = o;
+  return VDN_OK;
+}
+
 // The layer's launches in order: staging (fp32 narrowing / d padding, when
 // needed), Gram + inverse, scans, read-state packing, softmax kernel with the
 // merge epilogue. With `ev` set, ev[0..kProfileGroups] are recorded on the
@@ -406,7 +522,8 @@ constexpr int kProfileGroups = 5;
 
 int layer_launches(const Plan& P, const void* q, const void* k, const void* v, const void* kt,
                    const void* vt, const void* g_s, const void* g_l, const float* rms_w,
-                   void* out, uint8_t* ws, cudaStream_t st, cudaEvent_t* ev) {
+                   void* out, uint8_t* ws, cudaStream_t st, cudaEvent_t* ev,
+                   bool branches = false) {
   if (ev != nullptr) cudaEventRecord(ev[0], st);
   const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, true, true);
   if (ev != nullptr) cudaEventRecord(ev[1], st);
@@ -417,7 +534,7 @@ int layer_launches(const Plan& P, const void* q, const void* k, const void* v, c
   k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
                                                  ws + P.o_Rimg);
   if (ev != nullptr) cudaEventRecord(ev[4], st);
-  MergeArgs m{g_s, g_l, rms_w, out};
+  MergeArgs m{g_s, g_l, rms_w, out, branches};
   rc = launch_bsa(P, a, ws, nullptr, 0, kDPad, nullptr, st, &m);
   if (ev != nullptr) cudaEventRecord(ev[5], st);
   return rc;
@@ -489,6 +606,88 @@ int vdn_hybrid_attn_fwd_profile(const vdn_shape_t* shape, const void* q, const v
   for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
   delete[] ev;
   return rc;
+}
+
+size_t vdn_proj_workspace_bytes(const vdn_shape_t* shape, int D, int precision) {
+  Plan P;
+  ProjPlan Q;
+  if (make_plan(shape, &P) != VDN_OK || make_proj_plan(P, D, precision, &Q) != VDN_OK) return 0;
+  return Q.total;
+}
+
+int vdn_hybrid_attn_branches(const vdn_shape_t* shape, const void* q, const void* k,
+                             const void* v, const void* kt, const void* vt, const void* g_s,
+                             const void* g_l, const float* rms_w, void* branches,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (P.dtype != VDN_BF16 || P.d != kDPad) return VDN_ERR_UNSUPPORTED;
+  if (P.N == 0) return VDN_OK;
+  rc = check_ptrs({q, k, v, g_s, g_l, rms_w, branches}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  return finish(layer_launches(P, q, k, v, kt, vt, g_s, g_l, rms_w, branches,
+                               static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream),
+                               nullptr, true));
+}
+
+int vdn_linear(const void* a, const float* a_scale, const void* w, const float* w_scale,
+               int64_t M, int K, int D, int precision, void* y, void* stream) {
+  int rc = check_linear_args(a, a_scale, w, w_scale, M, K, D, precision, y);
+  if (rc != VDN_OK) return rc;
+  if (!set_smem_attrs() || !encode_fn()) return VDN_ERR_CUDA;
+  return finish(launch_linear(a, a_scale, w, w_scale, M, K, D, precision, y,
+                              static_cast<cudaStream_t>(stream)));
+}
+
+int vdn_quantize_rows_e4m3(const void* x, int64_t rows, int K, void* codes, float* scales,
+                           void* stream) {
+  if (rows < 0 || K < 16 || (K % 16) != 0 || rows > ((int64_t)1 << 31) - 1)
+    return VDN_ERR_INVALID_ARG;
+  if (rows == 0) return VDN_OK;
+  for (const void* p : {x, (const void*)codes, (const void*)scales}) {
+    if (p == nullptr) return VDN_ERR_INVALID_ARG;
+    if (!aligned16(p)) return VDN_ERR_MISALIGNED;
+  }
+  launch_quant(x, rows, K, codes, scales, static_cast<cudaStream_t>(stream));
+  return finish(VDN_OK);
+}
+
+int vdn_hybrid_attn_proj_fwd(const vdn_shape_t* shape, const void* q, const void* k,
+                             const void* v, const void* kt, const void* vt, const void* g_s,
+                             const void* g_l, const float* rms_w, const void* w_o,
+                             const float* w_scale, int D, int precision, void* y,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  ProjPlan Q;
+  rc = make_proj_plan(P, D, precision, &Q);
+  if (rc != VDN_OK) return rc;
+  if (P.N == 0) return VDN_OK;
+  rc = check_ptrs({q, k, v, g_s, g_l, rms_w, w_o, y}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  if (precision == VDN_PROJ_FP8 && (w_scale == nullptr || !aligned16(w_scale)))
+    return w_scale == nullptr ? VDN_ERR_INVALID_ARG : VDN_ERR_MISALIGNED;
+  if (workspace == nullptr || ws_bytes < Q.total) return VDN_ERR_WORKSPACE_TOO_SMALL;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* A = ws + Q.o_branches;
+  const int K = 2 * P.H * kDPad;
+  rc = layer_launches(P, q, k, v, kt, vt, g_s, g_l, rms_w, A, ws, st, nullptr, true);
+  if (rc != VDN_OK) return finish(rc);
+  if (precision == VDN_PROJ_FP8) {
+    float* sa = reinterpret_cast<float*>(ws + Q.o_scales);
+    launch_quant(A, P.N, K, ws + Q.o_codes, sa, st);
+    rc = launch_linear(ws + Q.o_codes, sa, w_o, w_scale, P.N, K, D, precision, y, st);
+  } else {
+    rc = launch_linear(A, nullptr, w_o, nullptr, P.N, K, D, precision, y, st);
+  }
+  return finish(rc);
 }
 
 int vdn_vda_scan(const vdn_shape_t* shape, const void* k, const void* v, const void* kt,
