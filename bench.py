@@ -399,6 +399,77 @@ def standalone_kernels(V, torch, w: Workload, stream, steps: int) -> dict:
     return dict(bsa_ms=t_bsa, merge_ms=t_merge)
 
 
+def projection_report(V, torch, w: Workload, stream, steps: int, peaks: dict) -> dict:
+    """The layer with per-branch output projections (w_o [H d, 2 H d],
+    synthetic weights): whole-layer ms in bf16 and e4m3, and the projection
+    GEMM and the activation quantiser timed alone."""
+    import vdn_synth as S
+    inp = w.inp
+    H, d, N = inp["H"], inp["d"], inp["N"]
+    D, K = H * d, 2 * H * d
+    w_bf = torch.from_numpy(S.make_proj_weight(H, d, seed=0)).to("cuda", torch.bfloat16)
+    w_codes = torch.empty((D, K), dtype=torch.uint8, device="cuda")
+    w_scale = torch.empty(D, dtype=torch.float32, device="cuda")
+    V.vdn_quantize_rows_e4m3(w_bf, D, K, w_codes, w_scale, stream)
+    y = torch.empty((N, D), dtype=torch.bfloat16, device="cuda")
+    dv = w.dev
+    rep = {"D": D, "K": K, "weights": "synthetic N(0,1)/sqrt(2Hd), bf16; e4m3 per output channel",
+           "gemm_tflop": round(2.0 * N * K * D / 1e12, 4)}
+    for prec, name in ((V.VDN_PROJ_BF16, "bf16"), (V.VDN_PROJ_FP8, "fp8")):
+        ws = V.alloc_proj_workspace(w.shape, D, prec)
+        wo, sc = (w_bf, None) if prec == V.VDN_PROJ_BF16 else (w_codes, w_scale)
+
+        def layer():
+            V.vdn_hybrid_attn_proj_fwd(w.shape, dv["q"], dv["k"], dv["v"], dv["kt"], dv["vt"],
+                                       dv["g_s"], dv["g_l"], w.rms_w, wo, sc, D, prec, y, ws,
+                                       stream)
+
+        layer()
+        time.sleep(REST_S)
+        t_layer = time_launches(torch, stream, layer, steps)
+        rep[f"layer_{name}_ms"] = round(t_layer, 4)
+        rep[f"layer_{name}_tflops"] = round((w.fl["total"] + 2.0 * N * K * D) / (t_layer * 1e-3)
+                                            / 1e12, 1)
+        del ws
+    # the GEMMs alone on the layer's own gated branches
+    br = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    ws = V.alloc_workspace(w.shape)
+    V.vdn_hybrid_attn_branches(w.shape, dv["q"], dv["k"], dv["v"], dv["kt"], dv["vt"], dv["g_s"],
+                               dv["g_l"], w.rms_w, br, ws, stream)
+    a_codes = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    a_scale = torch.empty(N, dtype=torch.float32, device="cuda")
+    V.vdn_quantize_rows_e4m3(br, N, K, a_codes, a_scale, stream)
+    flop = 2.0 * N * K * D
+    time.sleep(REST_S)
+    t_bf = time_launches(torch, stream, lambda: V.vdn_linear(br, None, w_bf, None, N, K, D,
+                                                             V.VDN_PROJ_BF16, y, stream), steps)
+    time.sleep(REST_S)
+    t_f8 = time_launches(torch, stream, lambda: V.vdn_linear(a_codes, a_scale, w_codes, w_scale, N,
+                                                             K, D, V.VDN_PROJ_FP8, y, stream), steps)
+    time.sleep(REST_S)
+    t_q = time_launches(torch, stream, lambda: V.vdn_quantize_rows_e4m3(br, N, K, a_codes, a_scale,
+                                                                        stream), steps)
+    qbytes = N * K * 2 + N * K + N * 4
+    rep["gemm_bf16"] = {"kernel": "k_linear<bf16>", "ms": round(t_bf, 4),
+                        "tflops": round(flop / (t_bf * 1e-3) / 1e12, 1),
+                        "frac": round(flop / (t_bf * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                        "peak": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']}"}
+    fp8_peak = 2 * peaks["bf16_tflops"]
+    rep["gemm_fp8"] = {"kernel": "k_linear<e4m3>", "ms": round(t_f8, 4),
+                       "tflops": round(flop / (t_f8 * 1e-3) / 1e12, 1),
+                       "frac": round(flop / (t_f8 * 1e-3) / 1e12 / fp8_peak, 4),
+                       "peak": f"2 x {peaks['source']} bf16 burst (nominal fp8/bf16 ratio) = "
+                               f"{fp8_peak}"}
+    rep["quant_e4m3"] = {"kernel": "k_quant_rows_e4m3", "ms": round(t_q, 4), "bytes": qbytes,
+                         "frac": round(qbytes / (t_q * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    del br, a_codes, ws
+    torch.cuda.synchronize()
+    rc = V.vdn_get_device_error()
+    if rc != 0:
+        raise RuntimeError(f"projections: {V.vdn_error_string(rc)}")
+    return rep
+
+
 def run_cuda(args) -> None:
     import torch
 
@@ -507,6 +578,9 @@ def run_cuda(args) -> None:
         if ww is not w:
             del ww
             torch.cuda.empty_cache()
+    proj = None
+    if not args.no_projections and w.inp["d"] == 128 and w.inp["dtype"] == "bf16":
+        proj = projection_report(V, torch, w, stream, args.steps, peaks)
     head = reports[args.workload]
     sm = head["softmax_merge"]
 
@@ -543,6 +617,8 @@ def run_cuda(args) -> None:
         "clocks": clocks,
         "workloads": reports,
     }
+    if proj is not None:
+        line["projections"] = proj
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w.inp, w.fl, args.workload, CPU_BASELINE_HEADS)
     if dist is not None:
@@ -688,6 +764,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-projections", action="store_true",
+                    help="skip the per-branch output projection measurements")
     ap.add_argument("--workloads", default="all", choices=["all", "none"],
                     help="also report every workload (default) or only the headline one")
     ap.add_argument("--profile", choices=["layer", "bsa", "vda", "merge"],
