@@ -337,8 +337,8 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
   bp.d_store = d_store;
   bp.lse = lse;
   bp.d = P.d;
-  // blocks on z (dispatched last), visited interior-first by the kernel
-  const dim3 grid((P.max_qtiles + 1) / 2, P.H, P.nb);
+  // heads on z (one head after the other), blocks on y visited interior-first
+  const dim3 grid((P.max_qtiles + 1) / 2, P.nb, P.H);
   if (merge == nullptr) {
     k_bsa_fwd<0><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
   } else {
