@@ -182,11 +182,11 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         const uint32_t sK = base + kBsaSmemK + (uint32_t)st * 32768u;
         const uint32_t sV = base + kBsaSmemV + (uint32_t)st * 32768u;
         const uint32_t kf = smem_u32(&bar_kf[st]), vf = smem_u32(&bar_vf[st]);
-        if (!mbar_wait_abortable(smem_u32(&bar_ke[st]), ph ^ 1, abort_v)) { *abort_v = 1; break; }
+        if (!mbar_wait(smem_u32(&bar_ke[st]), ph ^ 1)) { *abort_v = 1; break; }
         mbar_arrive_expect_tx(kf, 32768);
         tma_load_3d(sK, mk, kf, 0, h, row0);
         tma_load_3d(sK + 16384, mk, kf, 64, h, row0);
-        if (!mbar_wait_abortable(smem_u32(&bar_ve[st]), ph ^ 1, abort_v)) { *abort_v = 1; break; }
+        if (!mbar_wait(smem_u32(&bar_ve[st]), ph ^ 1)) { *abort_v = 1; break; }
         mbar_arrive_expect_tx(vf, 32768);
         tma_load_3d(sV, mv, vf, 0, h, row0);
         tma_load_3d(sV + 16384, mv, vf, 64, h, row0);
@@ -231,8 +231,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
                        sdesc_sw128(sQi + (uint32_t)((s >> 2) * 16384 + (s & 3) * 32), 16, 1024),
                        sdesc_sw128(sR + (uint32_t)(s * 2048), 16384, 1024), idO, s > 0 ? 1u : 0u);
       };
-      bool ok = mbar_wait_abortable(q_full, 0, abort_v) &&
-                mbar_wait_abortable(smem_u32(&bar_kf[0]), 0, abort_v);
+      bool ok = mbar_wait(q_full, 0) &&
+                mbar_wait(smem_u32(&bar_kf[0]), 0);
       if (ok) {
         tc_fence_after();
         qk(0, 0);
@@ -245,8 +245,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         const int st1 = (j + 1) & 1;
         const uint32_t ph1 = ((j + 1) >> 1) & 1;
         const bool more = j + 1 < nkt;
-        if (!mbar_wait_spin_abortable(smem_u32(&bar_vf[st]), ph, abort_v)) { ok = false; break; }
-        if (!mbar_wait_spin_abortable(smem_u32(&bar_pf[0]), (uint32_t)(j & 1), abort_v)) {
+        if (!mbar_wait_spin(smem_u32(&bar_vf[st]), ph)) { ok = false; break; }
+        if (!mbar_wait_spin(smem_u32(&bar_pf[0]), (uint32_t)(j & 1))) {
           ok = false;
           break;
         }
@@ -254,18 +254,18 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         pv(0, st, j > 0);
         if (!more) {
           if (kMerge) {
-            if (!mbar_wait_abortable(smem_u32(&bar_r), 0, abort_v)) { ok = false; break; }
+            if (!mbar_wait(smem_u32(&bar_r), 0)) { ok = false; break; }
             tc_fence_after();
             readout(0);
           }
           umma_commit(smem_u32(&bar_of[0]));
         }
         if (more) {
-          if (!mbar_wait_spin_abortable(smem_u32(&bar_kf[st1]), ph1, abort_v)) { ok = false; break; }
+          if (!mbar_wait_spin(smem_u32(&bar_kf[st1]), ph1)) { ok = false; break; }
           tc_fence_after();
           qk(0, st1);
         }
-        if (!mbar_wait_spin_abortable(smem_u32(&bar_pf[1]), (uint32_t)(j & 1), abort_v)) {
+        if (!mbar_wait_spin(smem_u32(&bar_pf[1]), (uint32_t)(j & 1))) {
           ok = false;
           break;
         }
@@ -303,11 +303,12 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     for (int j = 0; j < nkt; ++j) {
       int src, row0, valid;
       segs_tile(segs, j, src, row0, valid);
-      if (ok && !mbar_wait_abortable(s_full, (uint32_t)(j & 1), abort_v)) {
+      // no per-tile abort poll: a failed (bounded) wait ends the loop
+      if (!mbar_wait(s_full, (uint32_t)(j & 1))) {
         ok = false;
         *abort_v = 1;
+        break;
       }
-      if (ok) {
       tc_fence_after();
       uint32_t s[128];
       tmem_ld128(tS, s);
@@ -380,7 +381,6 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
-      }
     }
     const float l_sum = (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y) +
                         (lacc[2].x + lacc[2].y) + (lacc[3].x + lacc[3].y);
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
                         : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p.g_l)[gi]);
       }
     }
-    if (ok && !mbar_wait_abortable(smem_u32(&bar_of[tile]), 0, abort_v)) ok = false;
+    if (ok && !mbar_wait(smem_u32(&bar_of[tile]), 0)) ok = false;
     if (!ok) *abort_v = 1;
     tc_fence_after();
     const int row = qs + tile * kTile + r;

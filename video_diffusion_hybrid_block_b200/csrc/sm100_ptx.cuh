@@ -120,43 +120,6 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity) {
   }
 }
 
-// mbar_wait that also gives up, without recording an error, once another
-// role of the CTA has set *abort (after its own wait failed), so that one
-// failure ends every role's loop within one polling interval instead of one
-// wait limit per remaining iteration. *abort is read only while spinning.
-__device__ __forceinline__ bool mbar_wait_abortable(uint32_t bar, uint32_t parity,
-                                                    const volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        record_device_error(kDevErrWaitTimeout);
-        return false;
-      }
-    }
-  }
-}
-
-// Spinning variant of mbar_wait_abortable (test_wait, no suspend).
-__device__ __forceinline__ bool mbar_wait_spin_abortable(uint32_t bar, uint32_t parity,
-                                                         const volatile int* abort) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_test_wait(bar, parity)) return true;
-    if ((i & 255u) == 0) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        record_device_error(kDevErrWaitTimeout);
-        return false;
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------------ TMA --
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -506,12 +469,6 @@ __device__ __forceinline__ void regs_alloc() {
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// Arrive on a named barrier without waiting (the producer half of a
-// bar.arrive / bar.sync pair; nthreads counts both halves).
-__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Named barrier that also ANDs a predicate over the participating threads:
