@@ -1,9 +1,7 @@
 """The Gram kernel's inverse of M = lambda I + K^T K, emulated in float32 on
 the CPU: a 2 x 2 block inverse over 64 x 64 blocks through the Schur
-complement, whose two 64 x 64 inverses are block Gauss-Jordan sweeps with
-4 x 4 pivot blocks, without pivoting (M is SPD with eigenvalues >= lambda, so
-every pivot block is an SPD Schur complement); each 4 x 4 pivot block is
-inverted by scalar Gauss-Jordan.
+complement, whose two 64 x 64 inverses are Gauss-Jordan sweeps without
+pivoting (M is SPD with eigenvalues >= lambda, so every pivot is >= lambda).
 Checked against numpy's LU inverse on the key structures of the workloads:
 random keys, the low-rank keys of the hi-res workload (condition number in
 the hundreds), a single token (rank one) and no token (M = lambda I)."""
@@ -25,30 +23,13 @@ def gj(a):
     return a
 
 
-def block_gj(a, bs=4):
-    """In-place block Gauss-Jordan inverse with bs x bs pivot blocks, float32:
-    A_ij -= C_i P^-1 R_j, R_j <- P^-1 R_j, C_i <- -C_i P^-1, P <- P^-1."""
-    f = np.float32
-    a = np.asarray(a, f).copy()
-    for kb in range(a.shape[0] // bs):
-        k = slice(kb * bs, (kb + 1) * bs)
-        R, C = a[k, :].copy(), a[:, k].copy()
-        Pi = gj(R[:, k])
-        Q = (Pi @ R).astype(f)
-        a -= (C @ Q).astype(f)
-        a[k, :] = Q
-        a[:, k] = -(C @ Pi).astype(f)
-        a[k, k] = Pi
-    return a
-
-
 def block_inverse(M):
     f = np.float32
     M = np.asarray(M, f)
     A, B, D = M[:64, :64], M[:64, 64:], M[64:, 64:]
-    AI = block_gj(A)
+    AI = gj(A)
     X = (AI @ B).astype(f)
-    SI = block_gj((D - B.T @ X).astype(f))
+    SI = gj((D - B.T @ X).astype(f))
     Y = (X @ SI).astype(f)
     return np.block([[AI + Y @ X.T, -Y], [-Y.T, SI]]).astype(f)
 
@@ -76,13 +57,3 @@ def test_block_inverse_matches_lu(kind):
     assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-4
     # the symmetric inverse stays symmetric to rounding
     assert np.abs(got - got.T).max() < 1e-4 * np.abs(ref).max()
-
-
-def test_block_gj_equals_scalar_gj_to_rounding():
-    # the two sweeps compute the same inverse; block pivots change only the
-    # rounding order
-    rng = np.random.default_rng(3)
-    K = keys("random", rng)[:200]
-    A = (np.eye(128) + K.T @ K)[:64, :64]
-    a, b = gj(A).astype(np.float64), block_gj(A).astype(np.float64)
-    assert np.linalg.norm(a - b) / np.linalg.norm(a) < 1e-5

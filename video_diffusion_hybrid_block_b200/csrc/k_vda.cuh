@@ -17,11 +17,10 @@
 //   L2-normalises k rows in shared memory, accumulates G = K^T K and
 //   C^T = V^T K as two M=128 x N=128 bf16 tcgen05 contractions into TMEM,
 //   writes C^T (fp32, the layout the scan loads as its X operand)
-//   and then inverts M = lambda I + G (2 x 2 blocks of 64 through the Schur
-//   complement: two 64 x 64 block Gauss-Jordan sweeps in registers with
-//   4 x 4 pivot blocks, no pivoting since M is symmetric positive definite
-//   with eigenvalues >= lambda, and four 64^3 products) and writes
-//   W = M^-1 (fp32, tf32-rounded).
+//   and then inverts M = lambda I + G (2 x 2 blocks of 64: two 64-pivot
+//   Gauss-Jordan sweeps in registers, no pivoting since M is symmetric
+//   positive definite with eigenvalues >= lambda, and four 64^3 products
+//   through the Schur complement) and writes W = M^-1 (fp32, tf32-rounded).
 // Only frames whose state some block reads are processed: the forward scan
 //   stops at the largest forward read index, the backward scan at the
 //   smallest backward one (the remaining frames always sit inside the window
@@ -79,10 +78,8 @@ __global__ void __launch_bounds__(kGramThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_full[kGramStages], bar_empty[kGramStages], bar_done;
   __shared__ uint32_t tmem_slot;
-  // pivot row panel [4][64] and column panel [64][4] of the block
-  // Gauss-Jordan sweeps, double-buffered by step parity
-  __shared__ __align__(16) float rpan[2][4 * 64];
-  __shared__ __align__(16) float cpan[2][64 * 4];
+  __shared__ __align__(16) float rowbuf[2][128];
+  __shared__ __align__(16) float colbuf[2][128];
   __shared__ int abort_flag;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -237,10 +234,9 @@ __global__ void __launch_bounds__(kGramThreads, 2)
   // Inverse of M = lambda I + G = [[A, B], [B^T, D]] (64 x 64 blocks) by the
   // Schur complement: X = A^-1 B, S = D - B^T X, Y = X S^-1, and
   //   W = M^-1 = [[A^-1 + Y X^T, -Y], [-Y^T, S^-1]].
-  // A^-1 and S^-1 come from block Gauss-Jordan sweeps with 4 x 4 pivot
-  // blocks (no pivoting: both are symmetric positive definite with
-  // eigenvalues >= lambda) on 4 x 4 register tiles, thread (ty, tx) holding
-  // rows 4ty.., columns 4tx..; the
+  // A^-1 and S^-1 come from 64-pivot Gauss-Jordan sweeps (no pivoting: both
+  // are symmetric positive definite with eigenvalues >= lambda) on 4 x 4
+  // register tiles, thread (ty, tx) holding rows 4ty.., columns 4tx..; the
   // four 64 x 64 x 64 products are sums of rank-1 updates read from shared
   // memory as 16-byte vectors (A^-1 is symmetric; X and Y are also kept
   // transposed). W feeds only the scans' tf32 contractions and is stored
@@ -262,106 +258,45 @@ __global__ void __launch_bounds__(kGramThreads, 2)
   auto st4 = [](uint32_t addr, float x0, float x1, float x2, float x3) {
     st_shared_v4(addr, __float_as_uint(x0), __float_as_uint(x1), __float_as_uint(x2), __float_as_uint(x3));
   };
-  // In-place inverse of a 4 x 4 SPD block in registers (Gauss-Jordan, no
-  // pivoting: every pivot is a positive Schur complement).
-  auto inv4 = [](float (&q)[4][4]) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float ip;
-      asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(ip) : "f"(q[k][k]));
-      float rk[4], ck[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) rk[j] = q[k][j] * ip;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) ck[i] = q[i][k];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) q[i][j] = fmaf(-ck[i], rk[j], q[i][j]);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) q[k][j] = rk[j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) q[i][k] = -ck[i] * ip;
-      q[k][k] = ip;
-    }
-  };
-  // In-place Gauss-Jordan inverse of a 64 x 64 SPD matrix held in 4 x 4
-  // register tiles, four pivots per step (block Gauss-Jordan with 4 x 4
-  // pivot blocks, no pivoting: M is SPD, so every pivot block is an SPD
-  // Schur complement). Step kb, pivot block P = tile (kb, kb), pivot row
-  // panel R (tiles (kb, .)), pivot column panel C (tiles (., kb)):
-  //   A_ij -= C_i P^-1 R_j,  R_j <- P^-1 R_j,  C_i <- -C_i P^-1,  P <- P^-1.
-  // One block barrier per four pivots; every thread inverts P itself.
+  // in-place Gauss-Jordan inverse of a 64 x 64 SPD matrix held in 4 x 4 tiles
   auto gj64 = [&](float (&a)[4][4]) {
     for (int kb = 0; kb < 16; ++kb) {
-      float* rp = rpan[kb & 1];
-      float* cp = cpan[kb & 1];
-      if (ty == kb) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<float4*>(&rp[i * 64 + 4 * tx]) = make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
-      }
-      if (tx == kb) {
+      for (int kk = 0; kk < 4; ++kk) {
+        const int k = kb * 4 + kk;
+        const int buf = k & 1;
+        if (ty == kb)
+          *reinterpret_cast<float4*>(&rowbuf[buf][4 * tx]) = make_float4(a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
+        if (tx == kb)
+          *reinterpret_cast<float4*>(&colbuf[buf][4 * ty]) = make_float4(a[0][kk], a[1][kk], a[2][kk], a[3][kk]);
+        __syncthreads();
+        // pivot >= lambda > 0: the MUFU reciprocal (within a couple of ulp) is
+        // enough, and it shortens the per-pivot chain
+        float ip;
+        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(ip) : "f"(rowbuf[buf][k]));
+        const float4 r4 = *reinterpret_cast<const float4*>(&rowbuf[buf][4 * tx]);
+        const float4 c4 = *reinterpret_cast<const float4*>(&colbuf[buf][4 * ty]);
+        const float rj[4] = {r4.x * ip, r4.y * ip, r4.z * ip, r4.w * ip};
+        const float ci[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<float4*>(&cp[(4 * ty + i) * 4]) = make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
-      }
-      __syncthreads();
-      float pv[4][4], rj[4][4], ci[4][4];
+        for (int i = 0; i < 4; ++i) {
+          const float2 nc = make_float2(-ci[i], -ci[i]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 v = *reinterpret_cast<const float4*>(&rp[i * 64 + 4 * kb]);
-        pv[i][0] = v.x; pv[i][1] = v.y; pv[i][2] = v.z; pv[i][3] = v.w;
-        const float4 r4 = *reinterpret_cast<const float4*>(&rp[i * 64 + 4 * tx]);
-        rj[i][0] = r4.x; rj[i][1] = r4.y; rj[i][2] = r4.z; rj[i][3] = r4.w;
-        const float4 c4 = *reinterpret_cast<const float4*>(&cp[(4 * ty + i) * 4]);
-        ci[i][0] = c4.x; ci[i][1] = c4.y; ci[i][2] = c4.z; ci[i][3] = c4.w;
-      }
-      inv4(pv);
-      if (ty == kb && tx == kb) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) a[i][j] = pv[i][j];
-      } else if (tx == kb) {
-        // C_i <- -C_i P^-1
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float t = 0.f;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) t = fmaf(ci[i][k], pv[k][j], t);
-            a[i][j] = -t;
+          for (int j = 0; j < 4; j += 2) {
+            const float2 upd = ffma2(nc, make_float2(rj[j], rj[j + 1]), make_float2(a[i][j], a[i][j + 1]));
+            a[i][j] = upd.x;
+            a[i][j + 1] = upd.y;
           }
-      } else {
-        // Q = P^-1 R_j; the pivot row panel becomes Q, the rest A_ij - C_i Q
-        float qj[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float t = 0.f;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) t = fmaf(pv[i][k], rj[k][j], t);
-            qj[i][j] = t;
-          }
+        }
         if (ty == kb) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) a[i][j] = qj[i][j];
-        } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float t = a[i][j];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) t = fmaf(-ci[i][k], qj[k][j], t);
-              a[i][j] = t;
-            }
+          for (int j = 0; j < 4; ++j) a[kk][j] = rj[j];
         }
+        if (tx == kb) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a[i][kk] = -ci[i] * ip;
+        }
+        if (ty == kb && tx == kb) a[kk][kk] = ip;
       }
     }
   };
