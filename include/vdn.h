@@ -168,6 +168,36 @@ int vdn_hybrid_attn_proj_fwd(const vdn_shape_t* shape, const void* q, const void
                              const void* w_o, const float* w_scale, int D, int precision,
                              void* y, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * FP8 softmax branch. The pages pair FlashAttention-4 with FP8 on B200
+ * [agentlenshq.com page, core-ideas table; aigc.douyoubuy.cn page, section
+ * 07]. Reading implemented: QK^T and PV as e4m3 x e4m3 contractions with fp32
+ * accumulation; q has one scale per (token, head) row, k and v one scale per
+ * head over all video and text tokens (scale = amax / 448, codes rounded to
+ * nearest even in fp32); P is rounded to e4m3 after the exponential (P <= 256
+ * by the kernel's lazy rescale, so it needs no scale); the row sums use the
+ * unrounded P. Same shapes and layouts as vdn_bsa_fwd / vdn_hybrid_attn_fwd;
+ * bf16 activations with d = 128 only (VDN_ERR_UNSUPPORTED otherwise).
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes of the two entry points below (0 if unsupported): the
+ * layer's workspace plus the e4m3 codes of q, k, v, kt, vt, the q row scales,
+ * the per-head amax words and an o_soft buffer. */
+size_t vdn_fp8_workspace_bytes(const vdn_shape_t* shape);
+
+/* Softmax branch in e4m3: o_soft [N, H, d] bf16, lse [H, N] optional. */
+int vdn_bsa_fwd_fp8(const vdn_shape_t* shape, const void* q, const void* k, const void* v,
+                    const void* kt, const void* vt, void* o_soft, float* lse, void* workspace,
+                    size_t ws_bytes, void* stream);
+
+/* Whole layer with the e4m3 softmax branch; the linear branch, readout,
+ * RMSNorm and merge as in vdn_hybrid_attn_fwd (the merge runs as its own
+ * kernel on the e4m3 branch's o_soft). Writes out [N, H, d] bf16. */
+int vdn_hybrid_attn_fwd_fp8(const vdn_shape_t* shape, const void* q, const void* k,
+                            const void* v, const void* kt, const void* vt, const void* g_s,
+                            const void* g_l, const float* rms_w, void* out, void* workspace,
+                            size_t ws_bytes, void* stream);
+
 /* Measurement helper (no paper counterpart). Runs vdn_hybrid_attn_fwd (same
  * arguments) `iters` times (1..256) on `stream` with CUDA events recorded on
  * that stream between its kernels, waits for the stream, and writes the mean

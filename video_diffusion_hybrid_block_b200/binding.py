@@ -68,6 +68,10 @@ _SIGS = {
     "vdn_quantize_rows_e4m3": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int, _P, _P, _P]),
     "vdn_hybrid_attn_proj_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 8
                                  + [_P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _SZ, _P]),
+    "vdn_fp8_workspace_bytes": (_SZ, [ctypes.POINTER(vdn_shape_t)]),
+    "vdn_bsa_fwd_fp8": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
+    "vdn_hybrid_attn_fwd_fp8": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 9
+                                + [_P, _SZ, _P]),
     "vdn_vda_scan": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 8 + [_P, _SZ, _P]),
     "vdn_gate_merge": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
     "vdn_bsa_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
@@ -296,6 +300,42 @@ def vdn_selftest_wait_timeout(limit_ns: int, tmem_cols: int = 0, stream=None):
 
 def vdn_get_device_error() -> int:
     return int(load_library().vdn_get_device_error())
+
+
+# --------------------------------------------------- e4m3 softmax branch ---
+
+def vdn_fp8_workspace_bytes(shape: Shape) -> int:
+    return int(load_library().vdn_fp8_workspace_bytes(shape.ref))
+
+
+def alloc_fp8_workspace(shape: Shape, device=None) -> torch.Tensor:
+    n = vdn_fp8_workspace_bytes(shape)
+    if n == 0:
+        raise VdnError(VDN_ERR_UNSUPPORTED, "vdn_fp8_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def vdn_bsa_fwd_fp8(shape: Shape, q, k, v, kt, vt, o_soft, lse, workspace, stream=None,
+                    ws_bytes=None):
+    _check_acts(shape, q, k, v, kt, vt)
+    _need(o_soft, shape.N * shape.H * shape.d, 2, "o_soft")
+    _need(lse, shape.H * shape.N, 4, "lse")
+    rc = load_library().vdn_bsa_fwd_fp8(
+        shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(o_soft), _ptr(lse),
+        _ptr(workspace), _nbytes(workspace, ws_bytes), _stream(stream))
+    _check(rc, "vdn_bsa_fwd_fp8")
+    return o_soft
+
+
+def vdn_hybrid_attn_fwd_fp8(shape: Shape, q, k, v, kt, vt, g_s, g_l, rms_w, out, workspace,
+                            stream=None, ws_bytes=None):
+    _check_acts(shape, q, k, v, kt, vt, g_s, g_l, out)
+    _need(rms_w, shape.H * shape.d, 4, "rms_w")
+    rc = load_library().vdn_hybrid_attn_fwd_fp8(
+        shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(g_s), _ptr(g_l),
+        _ptr(rms_w), _ptr(out), _ptr(workspace), _nbytes(workspace, ws_bytes), _stream(stream))
+    _check(rc, "vdn_hybrid_attn_fwd_fp8")
+    return out
 
 
 # ------------------------------------------------ per-branch projections ---

@@ -90,19 +90,31 @@ struct BsaParams {
   int out_f32;
   int d;                 // real head dim
   int tma_out;           // out is bf16 [N][H][128]: full tiles leave through a TMA store
+  // e4m3 variant only: per-(token, head) q scales [N][H] and the per-head
+  // amax bit patterns of k and v ([2][H]; scale = amax / 448, 1 if zero)
+  const float* q_scale;
+  const uint32_t* kv_amax;
 };
 
 // kMode: 0 = softmax branch only (o_soft, lse); 1 = merged layer output;
 // 2 = the two gated branches written side by side for the per-branch output
 // projections (out is [N][2H][128] bf16: head h holds sigmoid(g_s) O / l,
 // head H + h holds sigmoid(g_l) w * o_lin / rms).
-template <int kMode>
+//
+// kFp8 (softmax branch only): q, k, v arrive as e4m3 codes ([rows][H][128]
+// bytes, one 128-byte swizzle row per token) with a scale per (token, head)
+// row of q and per head for k and v. QK^T and PV run as kind::f8f6f4
+// contractions (K32 steps), P is rounded to e4m3 (P <= 256 < 448 needs no
+// scale) and packed four per TMEM column, the q and k scales fold into each
+// row's exponent scale and the v scale into the final 1 / l.
+template <int kMode, bool kFp8 = false>
 __global__ void __launch_bounds__(kBsaThreads, 1)
     k_bsa_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkt,
               const __grid_constant__ CUtensorMap tvt, const __grid_constant__ CUtensorMap tout,
               const BsaParams p) {
   constexpr bool kMerge = kMode != 0;
+  static_assert(!kFp8 || kMode == 0, "the e4m3 variant computes the softmax branch only");
   const int pair = blockIdx.x, h = blockIdx.z;
   const int b = block_in_visit_order(blockIdx.y, num_blocks(p.F, p.bf));
   int q0, q1;
@@ -161,11 +173,17 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      mbar_arrive_expect_tx(q_full, 2 * 32768);
-      tma_load_3d(sQ, &tq, q_full, 0, h, qs);
-      tma_load_3d(sQ + 16384, &tq, q_full, 64, h, qs);
-      tma_load_3d(sQ + 32768, &tq, q_full, 0, h, qs + kTile);
-      tma_load_3d(sQ + 49152, &tq, q_full, 64, h, qs + kTile);
+      if constexpr (kFp8) {
+        mbar_arrive_expect_tx(q_full, 2 * 16384);
+        tma_load_3d(sQ, &tq, q_full, 0, h, qs);
+        tma_load_3d(sQ + 32768, &tq, q_full, 0, h, qs + kTile);
+      } else {
+        mbar_arrive_expect_tx(q_full, 2 * 32768);
+        tma_load_3d(sQ, &tq, q_full, 0, h, qs);
+        tma_load_3d(sQ + 16384, &tq, q_full, 64, h, qs);
+        tma_load_3d(sQ + 32768, &tq, q_full, 0, h, qs + kTile);
+        tma_load_3d(sQ + 49152, &tq, q_full, 64, h, qs + kTile);
+      }
       if (kMerge) {
         mbar_arrive_expect_tx(smem_u32(&bar_r), kRImageBytes);
         bulk_load(base + kBsaSmemR, p.rimg + ((int64_t)b * p.H + h) * kRImageBytes, kRImageBytes,
@@ -183,13 +201,23 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         const uint32_t sV = base + kBsaSmemV + (uint32_t)st * 32768u;
         const uint32_t kf = smem_u32(&bar_kf[st]), vf = smem_u32(&bar_vf[st]);
         if (!mbar_wait(smem_u32(&bar_ke[st]), ph ^ 1)) { *abort_v = 1; break; }
-        mbar_arrive_expect_tx(kf, 32768);
-        tma_load_3d(sK, mk, kf, 0, h, row0);
-        tma_load_3d(sK + 16384, mk, kf, 64, h, row0);
+        if constexpr (kFp8) {
+          mbar_arrive_expect_tx(kf, 16384);
+          tma_load_3d(sK, mk, kf, 0, h, row0);
+        } else {
+          mbar_arrive_expect_tx(kf, 32768);
+          tma_load_3d(sK, mk, kf, 0, h, row0);
+          tma_load_3d(sK + 16384, mk, kf, 64, h, row0);
+        }
         if (!mbar_wait(smem_u32(&bar_ve[st]), ph ^ 1)) { *abort_v = 1; break; }
-        mbar_arrive_expect_tx(vf, 32768);
-        tma_load_3d(sV, mv, vf, 0, h, row0);
-        tma_load_3d(sV + 16384, mv, vf, 64, h, row0);
+        if constexpr (kFp8) {
+          mbar_arrive_expect_tx(vf, 16384);
+          tma_load_3d(sV, mv, vf, 0, h, row0);
+        } else {
+          mbar_arrive_expect_tx(vf, 32768);
+          tma_load_3d(sV, mv, vf, 0, h, row0);
+          tma_load_3d(sV + 16384, mv, vf, 64, h, row0);
+        }
       }
     }
     __syncwarp();
@@ -198,16 +226,26 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, 128, false, false);
       const uint32_t idO = idesc_bf16(128, 128, false, true);
+      const uint32_t idS8 = idesc_e4m3(128, 128, false, false);
+      const uint32_t idO8 = idesc_e4m3(128, 128, false, true);
       // S_i = Q_i K^T for key tile in K stage st
       auto qk = [&](int i, int st) {
         const uint32_t sQi = sQ + (uint32_t)i * 32768u;
         const uint32_t sK = base + kBsaSmemK + (uint32_t)st * 32768u;
         const uint32_t dS = tmem + (uint32_t)(i * 128);
+        if constexpr (kFp8) {
+          // one 128-byte row per token: four K32 steps 32 bytes apart
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const uint32_t ko = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
-          umma_bf16_ss(dS, sdesc_sw128(sQi + ko, 16, 1024), sdesc_sw128(sK + ko, 16, 1024), idS,
-                       s > 0 ? 1u : 0u);
+          for (int s = 0; s < 4; ++s)
+            umma_f8_ss(dS, sdesc_sw128(sQi + (uint32_t)(s * 32), 16, 1024),
+                       sdesc_sw128(sK + (uint32_t)(s * 32), 16, 1024), idS8, s > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            const uint32_t ko = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
+            umma_bf16_ss(dS, sdesc_sw128(sQi + ko, 16, 1024), sdesc_sw128(sK + ko, 16, 1024), idS,
+                         s > 0 ? 1u : 0u);
+          }
         }
         umma_commit(smem_u32(&bar_sf[i]));
       };
@@ -216,10 +254,19 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         const uint32_t sV = base + kBsaSmemV + (uint32_t)st * 32768u;
         const uint32_t aP = tmem + (uint32_t)(i * 128);
         const uint32_t dO = tmem + 256u + (uint32_t)(i * 128);
+        if constexpr (kFp8) {
+          // P: four e4m3 per TMEM column (8 columns per K32 step); V MN-major,
+          // 32 key rows of 128 bytes per step
 #pragma unroll
-        for (int s = 0; s < 8; ++s)
-          umma_bf16_ts(dO, aP + (uint32_t)(s * 8), sdesc_sw128(sV + (uint32_t)(s * 2048), 16384, 1024),
-                       idO, (acc || s > 0) ? 1u : 0u);
+          for (int s = 0; s < 4; ++s)
+            umma_f8_ts(dO, aP + (uint32_t)(s * 8), sdesc_sw128(sV + (uint32_t)(s * 4096), 16384, 1024),
+                       idO8, (acc || s > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int s = 0; s < 8; ++s)
+            umma_bf16_ts(dO, aP + (uint32_t)(s * 8), sdesc_sw128(sV + (uint32_t)(s * 2048), 16384, 1024),
+                         idO, (acc || s > 0) ? 1u : 0u);
+        }
       };
       // o_lin_i = Q_i R_b into the S_i columns (merge variant, after PV_i's last tile)
       auto readout = [&](int i) {
@@ -295,7 +342,18 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     const uint32_t tO = tmem + lane_base + 256u + (uint32_t)(tile * 128);
     const uint32_t s_full = smem_u32(&bar_sf[tile]);
     const uint32_t p_full = smem_u32(&bar_pf[tile]);
-    const float scale = p.scale_log2;
+    float scale = p.scale_log2;
+    float v_scale = 1.f;
+    if constexpr (kFp8) {
+      // e4m3 scores are q8 . k8: fold the row's q scale and the head's k scale
+      // into the exponent scale, the head's v scale into 1 / l
+      const int qrow = qs + tile * kTile + r;
+      const float sq = qrow < q1 ? __ldg(p.q_scale + (int64_t)qrow * p.H + h) : 1.f;
+      const float ak = __uint_as_float(__ldg(p.kv_amax + h));
+      const float av = __uint_as_float(__ldg(p.kv_amax + p.H + h));
+      scale *= sq * (ak > 0.f ? __fdiv_rn(ak, 448.f) : 1.f);
+      v_scale = av > 0.f ? __fdiv_rn(av, 448.f) : 1.f;
+    }
     float m_use = 0.f;
     float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
@@ -363,6 +421,24 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       // first 64 TMEM columns
       const float2 sc2 = make_float2(scale, scale);
       const float2 nm2 = make_float2(-m_use, -m_use);
+      if constexpr (kFp8) {
+        // P as e4m3, four per TMEM column, into S_i's first 32 columns
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          const int c = 2 * e;
+          const float2 x0 = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2);
+          const float2 x1 = ffma2(make_float2(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])), sc2, nm2);
+          const float2 p0 = ((e & 3) == 3) ? exp2_poly2(x0)
+                                           : make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+          const float2 p1 = (((e + 1) & 3) == 3) ? exp2_poly2(x1)
+                                                 : make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+          lacc[e & 3] = fadd2(lacc[e & 3], p0);
+          lacc[(e + 1) & 3] = fadd2(lacc[(e + 1) & 3], p1);
+          pk[e >> 1] = e4m3x4(p0.x, p0.y, p1.x, p1.y);
+        }
+        tmem_st32(tS, pk);
+      } else {
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -377,6 +453,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
           pk[e] = pack_bf16x2(pe.x, pe.y);
         }
         tmem_st32(tS + (uint32_t)(half * 32), pk);
+      }
       }
       tmem_st_wait();
       tc_fence_before();
@@ -402,7 +479,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     tc_fence_after();
     const int row = qs + tile * kTile + r;
     const bool store = ok && row < q1;
-    const float inv = 1.f / l_sum;
+    const float inv = v_scale / l_sum;
     if (!kMerge) {
       __nv_bfloat16* dst = p.o + (int64_t)row * p.o_row_stride + (int64_t)h * p.d_store;
       // the TMEM loads are warp-collective: every thread runs them, only the

@@ -47,23 +47,6 @@ struct LinParams {
   const float* w_scale;   // e4m3 only: [D]
 };
 
-// Instruction descriptor, kind::f8f6f4 with e4m3 A/B (format 0) and f32 D,
-// same bit layout as idesc_bf16.
-__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
-  return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_f8_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
   asm volatile(
       "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
@@ -136,7 +119,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      const uint32_t idesc = kFp8 ? idesc_e4m3(kLinBM, kLinBN) : idesc_bf16(kLinBM, kLinBN, false, false);
+      const uint32_t idesc = kFp8 ? idesc_e4m3(kLinBM, kLinBN, false, false) : idesc_bf16(kLinBM, kLinBN, false, false);
       int it = 0, tl = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tl) {

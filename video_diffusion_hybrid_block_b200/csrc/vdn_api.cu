@@ -5,6 +5,7 @@
 // kernels.
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <initializer_list>
 #include <mutex>
@@ -15,6 +16,7 @@
 #include "k_linear.cuh"
 #include "k_merge.cuh"
 #include "k_prepare.cuh"
+#include "k_quant_attn.cuh"
 #include "k_vda.cuh"
 #include "layer_plan.cuh"
 #include "sm100_ptx.cuh"
@@ -50,6 +52,19 @@ bool map_act(CUtensorMap* m, const void* ptr, int64_t rows, int H, int box_rows)
   cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, H, 128] e4m3 codes as a 3-D tensor {128, H, rows}; box {128, 1, box_rows}.
+bool map_act8(CUtensorMap* m, const void* ptr, int64_t rows, int H, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kDPad, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)kDPad, (cuuint64_t)H * kDPad};
+  cuuint32_t box[3] = {128, 1, (cuuint32_t)box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -171,6 +186,8 @@ bool set_smem_attrs() {
                                  (int)kBsaSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_bsa_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBsaMergeSmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_bsa_fwd<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kBsaSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_bsa_fwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBsaMergeSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_linear<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -514,6 +531,99 @@ int make_proj_plan(const Plan& P, int D, int precision, ProjPlan* Q) {
   return VDN_OK;
 }
 
+// ------------------------------------------------------ e4m3 softmax --
+
+// Workspace of the e4m3 softmax branch: the layer's own workspace, then the
+// per-head amax words of k and v, the codes of q, k, v, kt, vt, the q row
+// scales and (for the whole layer) o_soft.
+struct Fp8Plan {
+  size_t o_amax, o_q8, o_k8, o_v8, o_kt8, o_vt8, o_qs, o_osoft, total;
+};
+
+int make_fp8_plan(const Plan& P, Fp8Plan* Q) {
+  if (P.dtype != VDN_BF16 || P.d != kDPad) return VDN_ERR_UNSUPPORTED;
+  const size_t act = (size_t)P.N * P.H * kDPad;
+  const size_t txt = (size_t)P.T * P.H * kDPad;
+  size_t o = P.total;
+  Q->o_amax = o; o += align256((size_t)2 * P.H * 4);
+  Q->o_q8 = o; o += align256(act);
+  Q->o_k8 = o; o += align256(act);
+  Q->o_v8 = o; o += align256(act);
+  Q->o_kt8 = o; o += align256(txt);
+  Q->o_vt8 = o; o += align256(txt);
+  Q->o_qs = o; o += align256((size_t)P.N * P.H * 4);
+  Q->o_osoft = o; o += align256(act * 2);
+  Q->total = o;
+  return VDN_OK;
+}
+
+int grid_for(int64_t units, int threads) {
+  return (int)std::min<int64_t>((units + threads - 1) / threads, (int64_t)148 * 8);
+}
+
+// amax of k, v per head (video and text together), then the e4m3 codes
+int launch_fp8_prepass(const Plan& P, const Fp8Plan& Q, const void* q, const void* k,
+                       const void* v, const void* kt, const void* vt, uint8_t* ws,
+                       cudaStream_t st) {
+  uint32_t* amax = reinterpret_cast<uint32_t*>(ws + Q.o_amax);
+  if (cudaMemsetAsync(amax, 0, (size_t)2 * P.H * 4, st) != cudaSuccess) return VDN_ERR_CUDA;
+  const int th = 256;
+  const auto bf = [](const void* x) { return static_cast<const __nv_bfloat16*>(x); };
+  if (P.N > 0) {
+    const int64_t u = (int64_t)P.N * P.H * 16;
+    k_attn_amax<<<grid_for(u, th), th, 0, st>>>(bf(k), bf(v), P.N, P.H, amax);
+  }
+  if (P.T > 0) {
+    const int64_t u = (int64_t)P.T * P.H * 16;
+    k_attn_amax<<<grid_for(u, th), th, 0, st>>>(bf(kt), bf(vt), P.T, P.H, amax);
+  }
+  if (P.N > 0) {
+    const int64_t u = (int64_t)P.N * P.H * 16;
+    k_attn_quant<<<grid_for(u, th), th, 0, st>>>(bf(q), bf(k), bf(v), P.N, P.H, amax,
+                                                ws + Q.o_q8, reinterpret_cast<float*>(ws + Q.o_qs),
+                                                ws + Q.o_k8, ws + Q.o_v8);
+  }
+  if (P.T > 0) {
+    const int64_t u = (int64_t)P.T * P.H * 16;
+    k_attn_quant<<<grid_for(u, th), th, 0, st>>>(nullptr, bf(kt), bf(vt), P.T, P.H, amax, nullptr,
+                                                nullptr, ws + Q.o_kt8, ws + Q.o_vt8);
+  }
+  return VDN_OK;
+}
+
+// e4m3 softmax branch: o [N, H, 128] bf16 (row stride o_row), lse optional
+int launch_bsa_fp8(const Plan& P, const Fp8Plan& Q, uint8_t* ws, __nv_bfloat16* o, int64_t o_row,
+                   float* lse, cudaStream_t st) {
+  if (P.N == 0) return VDN_OK;
+  CUtensorMap tq, tk, tv, tkt, tvt;
+  void* dummy = ws + Q.o_q8;  // never dereferenced for an empty text
+  const bool t = P.T > 0;
+  if (!map_act8(&tq, ws + Q.o_q8, P.N, P.H, 128) || !map_act8(&tk, ws + Q.o_k8, P.N, P.H, 128) ||
+      !map_act8(&tv, ws + Q.o_v8, P.N, P.H, 128) ||
+      !map_act8(&tkt, t ? ws + Q.o_kt8 : dummy, t ? P.T : 1, P.H, 128) ||
+      !map_act8(&tvt, t ? ws + Q.o_vt8 : dummy, t ? P.T : 1, P.H, 128))
+    return VDN_ERR_CUDA;
+  BsaParams bp;
+  memset(&bp, 0, sizeof(bp));
+  bp.off = P.off_dev;
+  bp.F = P.F;
+  bp.T = P.T;
+  bp.H = P.H;
+  bp.bf = P.bf;
+  bp.N = P.N;
+  bp.scale_log2 = 1.4426950408889634f / sqrtf((float)P.d);
+  bp.o = o;
+  bp.o_row_stride = o_row;
+  bp.d_store = kDPad;
+  bp.lse = lse;
+  bp.d = P.d;
+  bp.q_scale = reinterpret_cast<const float*>(ws + Q.o_qs);
+  bp.kv_amax = reinterpret_cast<const uint32_t*>(ws + Q.o_amax);
+  const dim3 grid((P.max_qtiles + 1) / 2, P.nb, P.H);
+  k_bsa_fwd<0, true><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tq, bp);
+  return VDN_OK;
+}
+
 // The layer's launches in order: staging (fp32 narrowing / d padding, when
 // needed), Gram + inverse, scans, read-state packing, softmax kernel with the
 // merge epilogue. With `ev` set, ev[0..kProfileGroups] are recorded on the
@@ -686,6 +796,69 @@ int vdn_hybrid_attn_proj_fwd(const vdn_shape_t* shape, const void* q, const void
     rc = launch_linear(ws + Q.o_codes, sa, w_o, w_scale, P.N, K, D, precision, y, st);
   } else {
     rc = launch_linear(A, nullptr, w_o, nullptr, P.N, K, D, precision, y, st);
+  }
+  return finish(rc);
+}
+
+size_t vdn_fp8_workspace_bytes(const vdn_shape_t* shape) {
+  Plan P;
+  Fp8Plan Q;
+  if (make_plan(shape, &P) != VDN_OK || make_fp8_plan(P, &Q) != VDN_OK) return 0;
+  return Q.total;
+}
+
+int vdn_bsa_fwd_fp8(const vdn_shape_t* shape, const void* q, const void* k, const void* v,
+                    const void* kt, const void* vt, void* o_soft, float* lse, void* workspace,
+                    size_t ws_bytes, void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  Fp8Plan Q;
+  rc = make_fp8_plan(P, &Q);
+  if (rc != VDN_OK) return rc;
+  if (P.N == 0) return VDN_OK;
+  rc = check_ptrs({q, k, v, o_soft}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  if (lse != nullptr && !aligned16(lse)) return VDN_ERR_MISALIGNED;
+  if (workspace == nullptr || ws_bytes < Q.total) return VDN_ERR_WORKSPACE_TOO_SMALL;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  rc = launch_fp8_prepass(P, Q, q, k, v, kt, vt, ws, st);
+  if (rc == VDN_OK)
+    rc = launch_bsa_fp8(P, Q, ws, static_cast<__nv_bfloat16*>(o_soft), (int64_t)P.H * kDPad, lse,
+                        st);
+  return finish(rc);
+}
+
+int vdn_hybrid_attn_fwd_fp8(const vdn_shape_t* shape, const void* q, const void* k,
+                            const void* v, const void* kt, const void* vt, const void* g_s,
+                            const void* g_l, const float* rms_w, void* out, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  Fp8Plan Q;
+  rc = make_fp8_plan(P, &Q);
+  if (rc != VDN_OK) return rc;
+  if (P.N == 0) return VDN_OK;
+  rc = check_ptrs({q, k, v, g_s, g_l, rms_w, out}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  if (workspace == nullptr || ws_bytes < Q.total) return VDN_ERR_WORKSPACE_TOO_SMALL;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  rc = launch_fp8_prepass(P, Q, q, k, v, kt, vt, ws, st);
+  const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, false, false);
+  if (rc == VDN_OK) rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr);
+  __nv_bfloat16* o_soft = reinterpret_cast<__nv_bfloat16*>(ws + Q.o_osoft);
+  if (rc == VDN_OK) rc = launch_bsa_fp8(P, Q, ws, o_soft, (int64_t)P.H * kDPad, nullptr, st);
+  if (rc == VDN_OK) {
+    const float* R = reinterpret_cast<const float*>(ws + P.o_R);
+    rc = launch_merge(P, a.q, R, R + (size_t)P.nb * P.H * 128 * 128, kDPad, o_soft,
+                      (int64_t)P.H * kDPad, kDPad, g_s, g_l, rms_w, out, ws, st);
   }
   return finish(rc);
 }
