@@ -470,6 +470,46 @@ def projection_report(V, torch, w: Workload, stream, steps: int, peaks: dict) ->
     return rep
 
 
+def fp8_report(V, torch, w: Workload, stream, steps: int, peaks: dict) -> dict:
+    """The e4m3 softmax branch and the layer with it: entry-point times (the
+    quantisation pre-pass included) beside the bf16 softmax-only kernel."""
+    d = w.dev
+    ws8 = V.alloc_fp8_workspace(w.shape)
+    o = torch.empty(d["q"].shape, dtype=torch.bfloat16, device="cuda")
+
+    def bsa8():
+        V.vdn_bsa_fwd_fp8(w.shape, d["q"], d["k"], d["v"], d["kt"], d["vt"], o, None, ws8, stream)
+
+    def layer8():
+        V.vdn_hybrid_attn_fwd_fp8(w.shape, d["q"], d["k"], d["v"], d["kt"], d["vt"], d["g_s"],
+                                  d["g_l"], w.rms_w, w.out, ws8, stream)
+
+    bsa8()
+    time.sleep(REST_S)
+    t_b = time_launches(torch, stream, bsa8, steps)
+    layer8()
+    time.sleep(REST_S)
+    t_l = time_launches(torch, stream, layer8, steps)
+    fl = w.fl
+    fp8_peak = 2 * peaks["bf16_tflops"]
+    del ws8, o
+    torch.cuda.synchronize()
+    rc = V.vdn_get_device_error()
+    if rc != 0:
+        raise RuntimeError(f"fp8: {V.vdn_error_string(rc)}")
+    return {
+        "softmax_fp8": {"entry": "vdn_bsa_fwd_fp8 (e4m3 pre-pass + k_bsa_fwd<e4m3>)",
+                        "ms": round(t_b, 4),
+                        "tflops": round(fl["softmax"] / (t_b * 1e-3) / 1e12, 1),
+                        "frac": round(fl["softmax"] / (t_b * 1e-3) / 1e12 / fp8_peak, 4),
+                        "peak": f"2 x {peaks['source']} bf16 burst (nominal fp8/bf16 ratio) = "
+                                f"{fp8_peak}"},
+        "layer_fp8": {"entry": "vdn_hybrid_attn_fwd_fp8", "ms": round(t_l, 4),
+                      "tflops": round(fl["total"] / (t_l * 1e-3) / 1e12, 1)},
+        "tolerance": "o_soft rel-L2 <= 0.06 vs the fp64 oracle (e4m3 operands)",
+    }
+
+
 def run_cuda(args) -> None:
     import torch
 
@@ -578,9 +618,10 @@ def run_cuda(args) -> None:
         if ww is not w:
             del ww
             torch.cuda.empty_cache()
-    proj = None
+    proj = fp8 = None
     if not args.no_projections and w.inp["d"] == 128 and w.inp["dtype"] == "bf16":
         proj = projection_report(V, torch, w, stream, args.steps, peaks)
+        fp8 = fp8_report(V, torch, w, stream, args.steps, peaks)
     head = reports[args.workload]
     sm = head["softmax_merge"]
 
@@ -619,6 +660,8 @@ def run_cuda(args) -> None:
     }
     if proj is not None:
         line["projections"] = proj
+    if fp8 is not None:
+        line["fp8"] = fp8
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w.inp, w.fl, args.workload, CPU_BASELINE_HEADS)
     if dist is not None:
