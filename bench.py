@@ -773,8 +773,28 @@ def run_profile(args) -> None:
     R = torch.empty((nb, inp["H"], inp["d"], inp["d"]), device="cuda")
     o_soft = torch.empty(dev["q"].shape, dtype=torch.bfloat16, device="cuda")
 
+    D, K = inp["H"] * inp["d"], 2 * inp["H"] * inp["d"]
+    if args.profile in ("proj", "proj8"):
+        w_bf = torch.from_numpy(S.make_proj_weight(inp["H"], inp["d"], seed=0)).to("cuda",
+                                                                                 torch.bfloat16)
+        w_codes = torch.empty((D, K), dtype=torch.uint8, device="cuda")
+        w_scale = torch.empty(D, dtype=torch.float32, device="cuda")
+        V.vdn_quantize_rows_e4m3(w_bf, D, K, w_codes, w_scale)
+        prec = V.VDN_PROJ_FP8 if args.profile == "proj8" else V.VDN_PROJ_BF16
+        wsp = V.alloc_proj_workspace(shape, D, prec)
+        y = torch.empty((inp["N"], D), dtype=torch.bfloat16, device="cuda")
+    if args.profile == "bsa8":
+        ws8 = V.alloc_fp8_workspace(shape)
+
     def once():
-        if args.profile == "layer":
+        if args.profile in ("proj", "proj8"):
+            wo, sc = (w_codes, w_scale) if args.profile == "proj8" else (w_bf, None)
+            V.vdn_hybrid_attn_proj_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"],
+                                       dev["g_s"], dev["g_l"], rms_w, wo, sc, D, prec, y, wsp)
+        elif args.profile == "bsa8":
+            V.vdn_bsa_fwd_fp8(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"], o_soft,
+                              None, ws8)
+        elif args.profile == "layer":
             V.vdn_hybrid_attn_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"],
                                   dev["g_s"], dev["g_l"], rms_w, out, ws)
         elif args.profile == "bsa":
@@ -811,7 +831,7 @@ def main():
                     help="skip the per-branch output projection measurements")
     ap.add_argument("--workloads", default="all", choices=["all", "none"],
                     help="also report every workload (default) or only the headline one")
-    ap.add_argument("--profile", choices=["layer", "bsa", "vda", "merge"],
+    ap.add_argument("--profile", choices=["layer", "bsa", "vda", "merge", "proj", "proj8", "bsa8"],
                     help="only run launches of one entry point (for ncu captures)")
     ap.add_argument("--workload", default=HEADLINE,
                     help="workload name (vdn_synth.CONFIGS); the default is the headline one")
