@@ -215,6 +215,29 @@ int vdn_hybrid_attn_fwd_profile(const vdn_shape_t* shape, const void* q, const v
                                 void* out, void* workspace, size_t ws_bytes, void* stream,
                                 int iters, float* kernel_ms);
 
+/* The layer split at the read states, so that the two branches can run on
+ * different GPUs (branch-specific placement: the pages place the softmax and
+ * the linear branch on different devices [openi.cn page, 主要功能 item 5;
+ * nav.superapi.store page, Main Features, Branch-Specific Parallelism]).
+ * vdn_vda_read_images runs the linear branch (Grams, inverses, scans) and
+ * writes R_b = Sfwd + Sbwd of every (block, head) as one 32 KB bf16 tile,
+ * [nb][H] tiles in the layout the fused readout loads; vdn_read_images_bytes
+ * gives the size (nb * H * 32768). vdn_bsa_merge_fwd runs the softmax branch
+ * with the readout, RMSNorm and gated merge in its epilogue, reading those
+ * tiles from `rimg` (device memory of the calling GPU: copy them there
+ * first). The two calls in a row equal vdn_hybrid_attn_fwd. Both take the
+ * workspace of vdn_workspace_bytes(shape). */
+size_t vdn_read_images_bytes(const vdn_shape_t* shape);
+
+int vdn_vda_read_images(const vdn_shape_t* shape, const void* k, const void* v,
+                        const void* kt, const void* vt, void* rimg, void* workspace,
+                        size_t ws_bytes, void* stream);
+
+int vdn_bsa_merge_fwd(const vdn_shape_t* shape, const void* q, const void* k, const void* v,
+                      const void* kt, const void* vt, const void* g_s, const void* g_l,
+                      const float* rms_w, const void* rimg, void* out, void* workspace,
+                      size_t ws_bytes, void* stream);
+
 /* Linear branch states only. read_states [nb, H, d, d] fp32 (required;
  * nb = ceil(F / block_frames)) gets R_b. Optional (NULL to skip):
  * text_state [H, d, d]; fwd_states [F, H, d, d] gets Sfwd[i] for

@@ -239,3 +239,19 @@ def test_proj_layer_checks(lib):
                                         need, 0) == B.VDN_ERR_UNSUPPORTED
     assert lib.vdn_hybrid_attn_branches(shape(dtype=1).ref, *([FAKE] * 9), FAKE, need, 0) == \
         B.VDN_ERR_UNSUPPORTED
+
+
+def test_split_layer_checks(lib):
+    s = shape()
+    need = V.vdn_workspace_bytes(s)
+    assert V.vdn_read_images_bytes(s) == 2 * 2 * 32768          # nb = 2 blocks, H = 2
+    assert lib.vdn_vda_read_images(s.ref, FAKE, FAKE, FAKE, FAKE, None, FAKE, need, 0) == \
+        B.VDN_ERR_INVALID_ARG
+    assert lib.vdn_vda_read_images(s.ref, FAKE, FAKE, FAKE, FAKE, FAKE_MIS, FAKE, need, 0) == \
+        B.VDN_ERR_MISALIGNED
+    assert lib.vdn_vda_read_images(s.ref, *([FAKE] * 5), FAKE, need - 1, 0) == \
+        B.VDN_ERR_WORKSPACE_TOO_SMALL
+    args = [FAKE] * 8
+    assert lib.vdn_bsa_merge_fwd(s.ref, *args, None, FAKE, FAKE, need, 0) == B.VDN_ERR_INVALID_ARG
+    assert lib.vdn_bsa_merge_fwd(s.ref, *args, FAKE, FAKE, FAKE, need - 1, 0) == \
+        B.VDN_ERR_WORKSPACE_TOO_SMALL

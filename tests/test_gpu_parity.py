@@ -284,3 +284,49 @@ def test_profile_entry_matches_layer():
     assert set(ms) == set(V.PROFILE_GROUPS)
     for k in ("gram_inv", "scan", "pack", "softmax_merge"):
         assert ms[k] > 0, k
+
+
+class _OneProcessPair:
+    """Both ranks of branch_parallel_forward in one process, one after the
+    other (linear rank first): send stores the tiles, recv copies them. No
+    kernel waits on another; this checks the device calls and buffers of the
+    split, not the transport."""
+
+    def __init__(self):
+        self.rank, self.sent = 1, None
+
+    def get_world_size(self):
+        return 2
+
+    def get_rank(self):
+        return self.rank
+
+    def send(self, t, dst):
+        self.sent = t.clone()
+
+    def recv(self, t, src):
+        t.copy_(self.sent)
+
+
+@pytest.mark.parametrize("name", ["mid", "d64-f32", "pages-scale"])
+def test_split_layer_equals_layer(name):
+    # vdn_vda_read_images + vdn_bsa_merge_fwd (through the branch-specific
+    # placement orchestrator) equal vdn_hybrid_attn_fwd bit for bit
+    import video_diffusion_hybrid_block_b200 as V
+    from video_diffusion_hybrid_block_b200.branch_parallel import branch_parallel_forward
+    from vdn_cases import make_shape
+    inp = S.make_inputs(name) if name in S.CONFIGS else _cases(name) if name != "mid" else mid_case(seed=41)
+    dev = device_inputs(inp)
+    ref = run_layer(inp, dev)
+    shape = make_shape(inp)
+    ws = V.alloc_workspace(shape)
+    rimg = torch.empty(V.vdn_read_images_bytes(shape), dtype=torch.uint8, device="cuda")
+    out = torch.full_like(dev["q"], float("nan"))
+    pair = _OneProcessPair()
+    assert branch_parallel_forward(pair, shape, dev, rimg, out, ws) is None   # linear rank
+    pair.rank = 0
+    rimg.zero_()                                       # the softmax rank's own buffer
+    got = branch_parallel_forward(pair, shape, dev, rimg, out, ws)
+    torch.cuda.synchronize()
+    assert V.vdn_get_device_error() == 0
+    assert torch.equal(got, ref)

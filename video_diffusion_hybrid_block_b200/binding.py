@@ -72,6 +72,9 @@ _SIGS = {
     "vdn_bsa_fwd_fp8": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
     "vdn_hybrid_attn_fwd_fp8": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 9
                                 + [_P, _SZ, _P]),
+    "vdn_read_images_bytes": (_SZ, [ctypes.POINTER(vdn_shape_t)]),
+    "vdn_vda_read_images": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 5 + [_P, _SZ, _P]),
+    "vdn_bsa_merge_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 10 + [_P, _SZ, _P]),
     "vdn_vda_scan": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 8 + [_P, _SZ, _P]),
     "vdn_gate_merge": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
     "vdn_bsa_fwd": (ctypes.c_int, [ctypes.POINTER(vdn_shape_t)] + [_P] * 7 + [_P, _SZ, _P]),
@@ -300,6 +303,37 @@ def vdn_selftest_wait_timeout(limit_ns: int, tmem_cols: int = 0, stream=None):
 
 def vdn_get_device_error() -> int:
     return int(load_library().vdn_get_device_error())
+
+
+# ------------------------------------------ layer split at the read states ---
+
+def vdn_read_images_bytes(shape: Shape) -> int:
+    return int(load_library().vdn_read_images_bytes(shape.ref))
+
+
+def vdn_vda_read_images(shape: Shape, k, v, kt, vt, rimg, workspace, stream=None, ws_bytes=None):
+    """Linear branch up to the packed read-state tiles (nb * H tiles of 32 KB)."""
+    _check_acts(shape, k=k, v=v, kt=kt, vt=vt)
+    _need(rimg, vdn_read_images_bytes(shape), 1, "rimg")
+    rc = load_library().vdn_vda_read_images(
+        shape.ref, _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(rimg), _ptr(workspace),
+        _nbytes(workspace, ws_bytes), _stream(stream))
+    _check(rc, "vdn_vda_read_images")
+    return rimg
+
+
+def vdn_bsa_merge_fwd(shape: Shape, q, k, v, kt, vt, g_s, g_l, rms_w, rimg, out, workspace,
+                      stream=None, ws_bytes=None):
+    """Softmax branch + fused readout / RMSNorm / gated merge on given read-state tiles."""
+    _check_acts(shape, q, k, v, kt, vt, g_s, g_l, out)
+    _need(rms_w, shape.H * shape.d, 4, "rms_w")
+    _need(rimg, vdn_read_images_bytes(shape), 1, "rimg")
+    rc = load_library().vdn_bsa_merge_fwd(
+        shape.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), _ptr(g_s), _ptr(g_l),
+        _ptr(rms_w), _ptr(rimg), _ptr(out), _ptr(workspace), _nbytes(workspace, ws_bytes),
+        _stream(stream))
+    _check(rc, "vdn_bsa_merge_fwd")
+    return out
 
 
 # --------------------------------------------------- e4m3 softmax branch ---
