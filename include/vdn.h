@@ -181,8 +181,8 @@ int vdn_hybrid_attn_proj_fwd(const vdn_shape_t* shape, const void* q, const void
  * ------------------------------------------------------------------------- */
 
 /* Workspace bytes of the two entry points below (0 if unsupported): the
- * layer's workspace plus the e4m3 codes of q, k, v, kt, vt, the q row scales,
- * the per-head amax words and an o_soft buffer. */
+ * layer's workspace plus the e4m3 codes of q, k, v, kt, vt, the q row scales
+ * and the per-head amax words. */
 size_t vdn_fp8_workspace_bytes(const vdn_shape_t* shape);
 
 /* Softmax branch in e4m3: o_soft [N, H, d] bf16, lse [H, N] optional. */
@@ -191,8 +191,9 @@ int vdn_bsa_fwd_fp8(const vdn_shape_t* shape, const void* q, const void* k, cons
                     size_t ws_bytes, void* stream);
 
 /* Whole layer with the e4m3 softmax branch; the linear branch, readout,
- * RMSNorm and merge as in vdn_hybrid_attn_fwd (the merge runs as its own
- * kernel on the e4m3 branch's o_soft). Writes out [N, H, d] bf16. */
+ * RMSNorm and gated merge as in vdn_hybrid_attn_fwd (readout and merge fused
+ * into the e4m3 softmax kernel's epilogue, the readout contraction on the
+ * bf16 q). Writes out [N, H, d] bf16. */
 int vdn_hybrid_attn_fwd_fp8(const vdn_shape_t* shape, const void* q, const void* k,
                             const void* v, const void* kt, const void* vt, const void* g_s,
                             const void* g_l, const float* rms_w, void* out, void* workspace,

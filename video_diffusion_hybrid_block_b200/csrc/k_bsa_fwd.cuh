@@ -69,6 +69,15 @@ constexpr uint32_t kBsaSmemR = 6 * 32768;       // packed R_b (merge variant), 3
 constexpr uint32_t kBsaSmemBytes = 6 * 32768 + 1024;       // + alignment slack
 constexpr uint32_t kBsaMergeSmemBytes = 7 * 32768 + 1024;
 constexpr uint32_t kRImageBytes = 32768;  // one packed R_b tile (bf16, 128B-swizzled MN-major)
+// e4m3 layout (16 KB tiles): Q8 tiles 0 and 1, K8 and V8 two stages each,
+// then (merge variant) the bf16 Q tiles of the readout, which also stage the
+// output tiles, and the packed R_b.
+constexpr uint32_t kBsa8SmemK = 2 * 16384;
+constexpr uint32_t kBsa8SmemV = 4 * 16384;
+constexpr uint32_t kBsa8SmemQb = 6 * 16384;
+constexpr uint32_t kBsa8SmemR = 6 * 16384 + 2 * 32768;
+constexpr uint32_t kBsa8SmemBytes = 6 * 16384 + 1024;
+constexpr uint32_t kBsa8MergeSmemBytes = kBsa8SmemR + 32768 + 1024;
 constexpr int kBsaRowsPerCta = 2 * kTile;
 
 struct BsaParams {
@@ -101,7 +110,7 @@ struct BsaParams {
 // projections (out is [N][2H][128] bf16: head h holds sigmoid(g_s) O / l,
 // head H + h holds sigmoid(g_l) w * o_lin / rms).
 //
-// kFp8 (softmax branch only): q, k, v arrive as e4m3 codes ([rows][H][128]
+// kFp8 (softmax branch, or with kMode 1 the merged layer output): q, k, v arrive as e4m3 codes ([rows][H][128]
 // bytes, one 128-byte swizzle row per token) with a scale per (token, head)
 // row of q and per head for k and v. QK^T and PV run as kind::f8f6f4
 // contractions (K32 steps), P is rounded to e4m3 (P <= 256 < 448 needs no
@@ -112,9 +121,15 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     k_bsa_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkt,
               const __grid_constant__ CUtensorMap tvt, const __grid_constant__ CUtensorMap tout,
-              const BsaParams p) {
+              const __grid_constant__ CUtensorMap tqb, const BsaParams p) {
   constexpr bool kMerge = kMode != 0;
-  static_assert(!kFp8 || kMode == 0, "the e4m3 variant computes the softmax branch only");
+  static_assert(!kFp8 || kMode <= 1, "the e4m3 variant has no gated-branches output");
+  // shared-memory layout: tile strides and offsets of the two variants
+  constexpr uint32_t kTileB = kFp8 ? 16384u : 32768u;          // Q / K / V tile bytes
+  constexpr uint32_t kOffK = kFp8 ? kBsa8SmemK : kBsaSmemK;
+  constexpr uint32_t kOffV = kFp8 ? kBsa8SmemV : kBsaSmemV;
+  constexpr uint32_t kOffQb = kFp8 ? kBsa8SmemQb : kBsaSmemQ;   // bf16 Q (readout, out staging)
+  constexpr uint32_t kOffR = kFp8 ? kBsa8SmemR : kBsaSmemR;
   const int pair = blockIdx.x, h = blockIdx.z;
   const int b = block_in_visit_order(blockIdx.y, num_blocks(p.F, p.bf));
   int q0, q1;
@@ -174,9 +189,18 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
       if constexpr (kFp8) {
-        mbar_arrive_expect_tx(q_full, 2 * 16384);
+        // e4m3 Q tiles; the merge variant's readout also needs Q in bf16
+        mbar_arrive_expect_tx(q_full, 2 * 16384 + (kMerge ? 2 * 32768 : 0));
         tma_load_3d(sQ, &tq, q_full, 0, h, qs);
-        tma_load_3d(sQ + 32768, &tq, q_full, 0, h, qs + kTile);
+        tma_load_3d(sQ + 16384, &tq, q_full, 0, h, qs + kTile);
+        if (kMerge) {
+          const uint32_t sQb = base + kOffQb;
+          tma_prefetch_desc(&tqb);
+          tma_load_3d(sQb, &tqb, q_full, 0, h, qs);
+          tma_load_3d(sQb + 16384, &tqb, q_full, 64, h, qs);
+          tma_load_3d(sQb + 32768, &tqb, q_full, 0, h, qs + kTile);
+          tma_load_3d(sQb + 49152, &tqb, q_full, 64, h, qs + kTile);
+        }
       } else {
         mbar_arrive_expect_tx(q_full, 2 * 32768);
         tma_load_3d(sQ, &tq, q_full, 0, h, qs);
@@ -186,7 +210,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       }
       if (kMerge) {
         mbar_arrive_expect_tx(smem_u32(&bar_r), kRImageBytes);
-        bulk_load(base + kBsaSmemR, p.rimg + ((int64_t)b * p.H + h) * kRImageBytes, kRImageBytes,
+        bulk_load(base + kOffR, p.rimg + ((int64_t)b * p.H + h) * kRImageBytes, kRImageBytes,
                   smem_u32(&bar_r));
       }
       for (int j = 0; j < nkt; ++j) {
@@ -197,8 +221,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         segs_tile(segs, j, src, row0, valid);
         const CUtensorMap* mk = src ? &tkt : &tk;
         const CUtensorMap* mv = src ? &tvt : &tv;
-        const uint32_t sK = base + kBsaSmemK + (uint32_t)st * 32768u;
-        const uint32_t sV = base + kBsaSmemV + (uint32_t)st * 32768u;
+        const uint32_t sK = base + kOffK + (uint32_t)st * kTileB;
+        const uint32_t sV = base + kOffV + (uint32_t)st * kTileB;
         const uint32_t kf = smem_u32(&bar_kf[st]), vf = smem_u32(&bar_vf[st]);
         if (!mbar_wait(smem_u32(&bar_ke[st]), ph ^ 1)) { *abort_v = 1; break; }
         if constexpr (kFp8) {
@@ -230,8 +254,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       const uint32_t idO8 = idesc_e4m3(128, 128, false, true);
       // S_i = Q_i K^T for key tile in K stage st
       auto qk = [&](int i, int st) {
-        const uint32_t sQi = sQ + (uint32_t)i * 32768u;
-        const uint32_t sK = base + kBsaSmemK + (uint32_t)st * 32768u;
+        const uint32_t sQi = sQ + (uint32_t)i * kTileB;
+        const uint32_t sK = base + kOffK + (uint32_t)st * kTileB;
         const uint32_t dS = tmem + (uint32_t)(i * 128);
         if constexpr (kFp8) {
           // one 128-byte row per token: four K32 steps 32 bytes apart
@@ -251,7 +275,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       };
       // O_i += P_i V with P_i read from the first 64 TMEM columns of S_i
       auto pv = [&](int i, int st, bool acc) {
-        const uint32_t sV = base + kBsaSmemV + (uint32_t)st * 32768u;
+        const uint32_t sV = base + kOffV + (uint32_t)st * kTileB;
         const uint32_t aP = tmem + (uint32_t)(i * 128);
         const uint32_t dO = tmem + 256u + (uint32_t)(i * 128);
         if constexpr (kFp8) {
@@ -270,8 +294,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       };
       // o_lin_i = Q_i R_b into the S_i columns (merge variant, after PV_i's last tile)
       auto readout = [&](int i) {
-        const uint32_t sQi = sQ + (uint32_t)i * 32768u;
-        const uint32_t sR = base + kBsaSmemR;
+        const uint32_t sQi = base + kOffQb + (uint32_t)i * 32768u;   // bf16 Q
+        const uint32_t sR = base + kOffR;
 #pragma unroll
         for (int s = 0; s < 8; ++s)
           umma_bf16_ss(tmem + (uint32_t)(i * 128),
@@ -523,7 +547,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       // a full tile of a bf16 d=128 output leaves through the (now idle) Q_i
       // buffer and one TMA store; otherwise each thread stores its row
       const bool via_tma = p.tma_out && (qs + tile * kTile + kTile <= q1);
-      const uint32_t stage = sQ + (uint32_t)tile * 32768u;
+      const uint32_t stage = base + kOffQb + (uint32_t)tile * 32768u;
       if constexpr (kMode == 2) {
         // pass 0: soft branch into head h, pass 1: linear branch into head H + h
 #pragma unroll 1

@@ -187,7 +187,9 @@ bool set_smem_attrs() {
   ok = ok && cudaFuncSetAttribute(k_bsa_fwd<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBsaMergeSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_bsa_fwd<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kBsaSmemBytes) == cudaSuccess;
+                                  (int)kBsa8SmemBytes) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(k_bsa_fwd<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kBsa8MergeSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_bsa_fwd<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBsaMergeSmemBytes) == cudaSuccess;
   ok = ok && cudaFuncSetAttribute(k_linear<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -358,7 +360,7 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
   // heads on z (one head after the other), blocks on y visited interior-first
   const dim3 grid((P.max_qtiles + 1) / 2, P.nb, P.H);
   if (merge == nullptr) {
-    k_bsa_fwd<0><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
+    k_bsa_fwd<0><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, tq, bp);
   } else {
     bp.rimg = merge->rimg != nullptr ? merge->rimg : ws + P.o_Rimg;
     bp.g_s = merge->g_s;
@@ -370,9 +372,11 @@ int launch_bsa(const Plan& P, const Acts& a, uint8_t* ws, __nv_bfloat16* o, int6
     bp.out_f32 = (P.dtype == VDN_F32);
     bp.tma_out = tma_out ? 1 : 0;
     if (merge->branches)
-      k_bsa_fwd<2><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
+      k_bsa_fwd<2><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, tq,
+                                                                bp);
     else
-      k_bsa_fwd<1><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, bp);
+      k_bsa_fwd<1><<<grid, kBsaThreads, kBsaMergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout, tq,
+                                                                bp);
   }
   return VDN_OK;
 }
@@ -535,10 +539,10 @@ int make_proj_plan(const Plan& P, int D, int precision, ProjPlan* Q) {
 // ------------------------------------------------------ e4m3 softmax --
 
 // Workspace of the e4m3 softmax branch: the layer's own workspace, then the
-// per-head amax words of k and v, the codes of q, k, v, kt, vt, the q row
-// scales and (for the whole layer) o_soft.
+// per-head amax words of k and v, the codes of q, k, v, kt, vt and the q row
+// scales.
 struct Fp8Plan {
-  size_t o_amax, o_q8, o_k8, o_v8, o_kt8, o_vt8, o_qs, o_osoft, total;
+  size_t o_amax, o_q8, o_k8, o_v8, o_kt8, o_vt8, o_qs, total;
 };
 
 int make_fp8_plan(const Plan& P, Fp8Plan* Q) {
@@ -553,7 +557,6 @@ int make_fp8_plan(const Plan& P, Fp8Plan* Q) {
   Q->o_kt8 = o; o += align256(txt);
   Q->o_vt8 = o; o += align256(txt);
   Q->o_qs = o; o += align256((size_t)P.N * P.H * 4);
-  Q->o_osoft = o; o += align256(act * 2);
   Q->total = o;
   return VDN_OK;
 }
@@ -592,17 +595,23 @@ int launch_fp8_prepass(const Plan& P, const Fp8Plan& Q, const void* q, const voi
   return VDN_OK;
 }
 
-// e4m3 softmax branch: o [N, H, 128] bf16 (row stride o_row), lse optional
+// e4m3 softmax branch: o [N, H, 128] bf16 (row stride o_row), lse optional;
+// with `merge` set, the merged layer output instead (readout, RMSNorm and
+// gated merge in the epilogue, R_b tiles at ws + o_Rimg, q in bf16 `qb`).
 int launch_bsa_fp8(const Plan& P, const Fp8Plan& Q, uint8_t* ws, __nv_bfloat16* o, int64_t o_row,
-                   float* lse, cudaStream_t st) {
+                   float* lse, cudaStream_t st, const MergeArgs* merge = nullptr,
+                   const void* qb = nullptr) {
   if (P.N == 0) return VDN_OK;
-  CUtensorMap tq, tk, tv, tkt, tvt;
+  CUtensorMap tq, tk, tv, tkt, tvt, tout, tqb;
   void* dummy = ws + Q.o_q8;  // never dereferenced for an empty text
   const bool t = P.T > 0;
   if (!map_act8(&tq, ws + Q.o_q8, P.N, P.H, 128) || !map_act8(&tk, ws + Q.o_k8, P.N, P.H, 128) ||
       !map_act8(&tv, ws + Q.o_v8, P.N, P.H, 128) ||
       !map_act8(&tkt, t ? ws + Q.o_kt8 : dummy, t ? P.T : 1, P.H, 128) ||
       !map_act8(&tvt, t ? ws + Q.o_vt8 : dummy, t ? P.T : 1, P.H, 128))
+    return VDN_ERR_CUDA;
+  if (merge != nullptr && (!map_act(&tout, merge->out, P.N, P.H, 128) ||
+                           !map_act(&tqb, qb, P.N, P.H, 128)))
     return VDN_ERR_CUDA;
   BsaParams bp;
   memset(&bp, 0, sizeof(bp));
@@ -621,7 +630,21 @@ int launch_bsa_fp8(const Plan& P, const Fp8Plan& Q, uint8_t* ws, __nv_bfloat16* 
   bp.q_scale = reinterpret_cast<const float*>(ws + Q.o_qs);
   bp.kv_amax = reinterpret_cast<const uint32_t*>(ws + Q.o_amax);
   const dim3 grid((P.max_qtiles + 1) / 2, P.nb, P.H);
-  k_bsa_fwd<0, true><<<grid, kBsaThreads, kBsaSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tq, bp);
+  if (merge == nullptr) {
+    k_bsa_fwd<0, true><<<grid, kBsaThreads, kBsa8SmemBytes, st>>>(tq, tk, tv, tkt, tvt, tq, tq, bp);
+  } else {
+    bp.rimg = ws + P.o_Rimg;
+    bp.g_s = merge->g_s;
+    bp.g_l = merge->g_l;
+    bp.gate_f32 = 0;
+    bp.rms_w = merge->rms_w;
+    bp.eps = P.eps;
+    bp.out = merge->out;
+    bp.out_f32 = 0;
+    bp.tma_out = 1;
+    k_bsa_fwd<1, true><<<grid, kBsaThreads, kBsa8MergeSmemBytes, st>>>(tq, tk, tv, tkt, tvt, tout,
+                                                                       tqb, bp);
+  }
   return VDN_OK;
 }
 
@@ -854,61 +877,14 @@ int vdn_hybrid_attn_fwd_fp8(const vdn_shape_t* shape, const void* q, const void*
   rc = launch_fp8_prepass(P, Q, q, k, v, kt, vt, ws, st);
   const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, false, false);
   if (rc == VDN_OK) rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr);
-  __nv_bfloat16* o_soft = reinterpret_cast<__nv_bfloat16*>(ws + Q.o_osoft);
-  if (rc == VDN_OK) rc = launch_bsa_fp8(P, Q, ws, o_soft, (int64_t)P.H * kDPad, nullptr, st);
   if (rc == VDN_OK) {
     const float* R = reinterpret_cast<const float*>(ws + P.o_R);
-    rc = launch_merge(P, a.q, R, R + (size_t)P.nb * P.H * 128 * 128, kDPad, o_soft,
-                      (int64_t)P.H * kDPad, kDPad, g_s, g_l, rms_w, out, ws, st);
+    k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
+                                                   ws + P.o_Rimg);
+    MergeArgs m{g_s, g_l, rms_w, out};
+    rc = launch_bsa_fp8(P, Q, ws, nullptr, 0, nullptr, st, &m, q);
   }
   return finish(rc);
-}
-
-size_t vdn_read_images_bytes(const vdn_shape_t* shape) {
-  Plan P;
-  if (make_plan(shape, &P) != VDN_OK) return 0;
-  return (size_t)P.nb * P.H * kRImageBytes;
-}
-
-int vdn_vda_read_images(const vdn_shape_t* shape, const void* k, const void* v, const void* kt,
-                        const void* vt, void* rimg, void* workspace, size_t ws_bytes,
-                        void* stream) {
-  Plan P;
-  int rc = make_plan(shape, &P);
-  if (rc != VDN_OK) return rc;
-  if (P.N > 0) rc = check_ptrs({k, v, rimg}, {kt, vt}, P.T);
-  else rc = check_ptrs({rimg}, {kt, vt}, P.T);
-  if (rc != VDN_OK) return rc;
-  rc = common_checks(P, workspace, ws_bytes);
-  if (rc != VDN_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const Acts a = stage_inputs(P, nullptr, k, v, kt, vt, ws, st, false, true);
-  rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr);
-  if (rc != VDN_OK) return finish(rc);
-  const float* R = reinterpret_cast<const float*>(ws + P.o_R);
-  k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
-                                                 static_cast<uint8_t*>(rimg));
-  return finish(VDN_OK);
-}
-
-int vdn_bsa_merge_fwd(const vdn_shape_t* shape, const void* q, const void* k, const void* v,
-                      const void* kt, const void* vt, const void* g_s, const void* g_l,
-                      const float* rms_w, const void* rimg, void* out, void* workspace,
-                      size_t ws_bytes, void* stream) {
-  Plan P;
-  int rc = make_plan(shape, &P);
-  if (rc != VDN_OK) return rc;
-  if (P.N == 0) return VDN_OK;
-  rc = check_ptrs({q, k, v, g_s, g_l, rms_w, rimg, out}, {kt, vt}, P.T);
-  if (rc != VDN_OK) return rc;
-  rc = common_checks(P, workspace, ws_bytes);
-  if (rc != VDN_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, true, true);
-  MergeArgs m{g_s, g_l, rms_w, out, false, static_cast<const uint8_t*>(rimg)};
-  return finish(launch_bsa(P, a, ws, nullptr, 0, kDPad, nullptr, st, &m));
 }
 
 int vdn_vda_scan(const vdn_shape_t* shape, const void* k, const void* v, const void* kt,
