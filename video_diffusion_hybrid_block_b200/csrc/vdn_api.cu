@@ -887,6 +887,53 @@ int vdn_hybrid_attn_fwd_fp8(const vdn_shape_t* shape, const void* q, const void*
   return finish(rc);
 }
 
+size_t vdn_read_images_bytes(const vdn_shape_t* shape) {
+  Plan P;
+  if (make_plan(shape, &P) != VDN_OK) return 0;
+  return (size_t)P.nb * P.H * kRImageBytes;
+}
+
+int vdn_vda_read_images(const vdn_shape_t* shape, const void* k, const void* v, const void* kt,
+                        const void* vt, void* rimg, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (P.N > 0) rc = check_ptrs({k, v, rimg}, {kt, vt}, P.T);
+  else rc = check_ptrs({rimg}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const Acts a = stage_inputs(P, nullptr, k, v, kt, vt, ws, st, false, true);
+  rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr);
+  if (rc != VDN_OK) return finish(rc);
+  const float* R = reinterpret_cast<const float*>(ws + P.o_R);
+  k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
+                                                 static_cast<uint8_t*>(rimg));
+  return finish(VDN_OK);
+}
+
+int vdn_bsa_merge_fwd(const vdn_shape_t* shape, const void* q, const void* k, const void* v,
+                      const void* kt, const void* vt, const void* g_s, const void* g_l,
+                      const float* rms_w, const void* rimg, void* out, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  Plan P;
+  int rc = make_plan(shape, &P);
+  if (rc != VDN_OK) return rc;
+  if (P.N == 0) return VDN_OK;
+  rc = check_ptrs({q, k, v, g_s, g_l, rms_w, rimg, out}, {kt, vt}, P.T);
+  if (rc != VDN_OK) return rc;
+  rc = common_checks(P, workspace, ws_bytes);
+  if (rc != VDN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const Acts a = stage_inputs(P, q, k, v, kt, vt, ws, st, true, true);
+  MergeArgs m{g_s, g_l, rms_w, out, false, static_cast<const uint8_t*>(rimg)};
+  return finish(launch_bsa(P, a, ws, nullptr, 0, kDPad, nullptr, st, &m));
+}
+
 int vdn_vda_scan(const vdn_shape_t* shape, const void* k, const void* v, const void* kt,
                  const void* vt, float* read_states, float* text_state, float* fwd_states,
                  float* bwd_states, void* workspace, size_t ws_bytes, void* stream) {
