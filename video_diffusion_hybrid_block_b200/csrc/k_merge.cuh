@@ -222,7 +222,8 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
 // contraction) and leaves through one TMA store; a block's ragged last tile
 // is stored row by row. Hand-offs: in_full/in_empty per stage, acc_full /
 // acc_empty per TMEM buffer.
-constexpr int kMergeTmaThreads = 160;
+constexpr int kMergeTmaThreads = 288;          // 8 epilogue warps + the load / MMA warp
+constexpr int kMergeTmaEpi = 256;
 constexpr int kMergeTmaStages = 3;
 constexpr int kMergeTmaTiles = 14;           // 3 CTAs cover a 40-tile block
 constexpr uint32_t kMergeTmaSmemR = 0;       // 32 KB
@@ -244,6 +245,7 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
   __shared__ uint64_t in_full[kMergeTmaStages], in_empty[kMergeTmaStages], acc_full[2], acc_empty[2];
   __shared__ uint32_t tmem_slot;
   __shared__ float wsm[128];
+  __shared__ float ssh[2][128];  // per-row sums of squares of the two column halves
   __shared__ int abort_flag;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sR = base + kMergeTmaSmemR;
@@ -273,9 +275,9 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
   const uint32_t tmem = tmem_slot;
   volatile int* abort_v = &abort_flag;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------ loads and contractions
-    if (i == 128) {
+    if (i == kMergeTmaEpi) {
       auto load_tile = [&](int t) {
         const int st = t % kMergeTmaStages;
         const uint32_t bar = smem_u32(&in_full[st]);
@@ -293,7 +295,7 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
     }
     // R_b is ready once the epilogue warps pass this barrier
     named_barrier_sync(1, kMergeTmaThreads);
-    if (i == 128) {
+    if (i == kMergeTmaEpi) {
       const uint32_t idO = idesc_bf16(128, 128, false, true);
       for (int t = 0; t < ntl; ++t) {
         if (*abort_v) break;
@@ -334,34 +336,39 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    // R_b (fwd + bwd) -> bf16, row i (key dim), MN-major 128B-swizzled
-    const int64_t rbase = ((int64_t)b * p.H + h) * 128 * 128;
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
+    // 8 warps: warp w reads TMEM lane quarter w % 4 (rows 32 (w % 4) ..) and
+    // column half w / 4; the RMSNorm sum of squares of a row is the sum of
+    // its two halves, exchanged through shared memory.
+    // R_b (fwd + bwd) -> bf16, MN-major 128B-swizzled: thread i converts
+    // chunk i / 128 (64 value dims) of row i % 128 (key dim)
+    {
+      const int rr = i & 127, c = i >> 7;
+      const int64_t rbase = ((int64_t)b * p.H + h) * 128 * 128;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const float4* ra = reinterpret_cast<const float4*>(p.RA + rbase + (int64_t)i * 128 + c * 64 + u * 8);
+        const float4* ra = reinterpret_cast<const float4*>(p.RA + rbase + (int64_t)rr * 128 + c * 64 + u * 8);
         float4 x0 = __ldg(ra), x1 = __ldg(ra + 1);
         if (p.RB) {
-          const float4* rb = reinterpret_cast<const float4*>(p.RB + rbase + (int64_t)i * 128 + c * 64 + u * 8);
+          const float4* rb = reinterpret_cast<const float4*>(p.RB + rbase + (int64_t)rr * 128 + c * 64 + u * 8);
           const float4 y0 = __ldg(rb), y1 = __ldg(rb + 1);
           x0 = make_float4(x0.x + y0.x, x0.y + y0.y, x0.z + y0.z, x0.w + y0.w);
           x1 = make_float4(x1.x + y1.x, x1.y + y1.y, x1.z + y1.z, x1.w + y1.w);
         }
-        st_shared_v4(sR + (uint32_t)(c * 16384) + sw128_off((uint32_t)i, (uint32_t)u),
+        st_shared_v4(sR + (uint32_t)(c * 16384) + sw128_off((uint32_t)rr, (uint32_t)u),
                      pack_bf16x2(x0.x, x0.y), pack_bf16x2(x0.z, x0.w), pack_bf16x2(x1.x, x1.y),
                      pack_bf16x2(x1.z, x1.w));
       }
     }
-    wsm[i] = __ldg(p.rms_w + (int64_t)h * 128 + i);
+    if (i < 128) wsm[i] = __ldg(p.rms_w + (int64_t)h * 128 + i);
     fence_proxy_async_smem();
     named_barrier_sync(1, kMergeTmaThreads);
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + (i & 31);   // row of the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     for (int t = 0; t < ntl; ++t) {
-      if (*abort_v) break;
       const int st = t % kMergeTmaStages, ab = t & 1;
       const int row0 = q0 + (t_first + t) * kTile;
-      const int row = row0 + i;
+      const int row = row0 + r;
       const bool valid = row < q1;
       const bool full_tile = row0 + kTile <= q1;
       float gsv = 0.f, glv = 0.f;
@@ -369,37 +376,43 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
         gsv = sigmoidf_(load_gate(p.g_s, (int64_t)row * p.H + h, p.gate_f32));
         glv = sigmoidf_(load_gate(p.g_l, (int64_t)row * p.H + h, p.gate_f32));
       }
-      if (!mbar_wait(smem_u32(&acc_full[ab]), (uint32_t)((t >> 1) & 1))) { *abort_v = 1; break; }
+      const bool mine = !*abort_v && mbar_wait(smem_u32(&acc_full[ab]), (uint32_t)((t >> 1) & 1));
+      // uniform over the 256 epilogue threads: all leave or none does
+      if (!named_barrier_and(2, kMergeTmaEpi, mine)) {
+        *abort_v = 1;
+        break;
+      }
       tc_fence_after();
-      const uint32_t tO = tmem + lane_base + (uint32_t)(ab * 128);
+      const uint32_t tO = tmem + lane_base + (uint32_t)(ab * 128 + half * 64);
+      uint32_t o[2][32];
+      tmem_ld32(tO, o[0]);
+      tmem_ld32(tO + 32u, o[1]);
+      tmem_ld_wait(o[0]);
+      tmem_ld_wait(o[1]);
       float ss = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + (uint32_t)(c * 32), o);
-        tmem_ld_wait(o);
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(o[e]), __uint_as_float(o[e]), ss);
-      }
+        for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(o[c][e]), __uint_as_float(o[c][e]), ss);
+      ssh[half][r] = ss;
+      named_barrier_sync(2, kMergeTmaEpi);
+      ss = ssh[0][r] + ssh[1][r];
       const float nr = glv * rsqrtf(ss * (1.f / 128.f) + p.eps);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + ((int64_t)row * p.H + h) * 128;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + (uint32_t)(c * 32), o);
-        tmem_ld_wait(o);
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int c0 = c * 32 + u * 8;
-          const uint32_t off = (uint32_t)(c0 >> 6) * 16384u + sw128_off((uint32_t)i, (uint32_t)((c0 & 63) >> 3));
+          const int c0 = half * 64 + c * 32 + u * 8;
+          const uint32_t off = (uint32_t)half * 16384u + sw128_off((uint32_t)r, (uint32_t)((c0 & 63) >> 3));
           const uint4 ov = ld_shared_v4(sO(st) + off);
           const uint32_t w4[4] = {ov.x, ov.y, ov.z, ov.w};
           uint32_t y4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int cc = c0 + 2 * e;
-            const float ylo = gsv * bf_lo(w4[e]) + nr * wsm[cc] * __uint_as_float(o[u * 8 + 2 * e]);
-            const float yhi = gsv * bf_hi(w4[e]) + nr * wsm[cc + 1] * __uint_as_float(o[u * 8 + 2 * e + 1]);
+            const float ylo = gsv * bf_lo(w4[e]) + nr * wsm[cc] * __uint_as_float(o[c][u * 8 + 2 * e]);
+            const float yhi = gsv * bf_hi(w4[e]) + nr * wsm[cc + 1] * __uint_as_float(o[c][u * 8 + 2 * e + 1]);
             y4[e] = pack_bf16x2(ylo, yhi);
           }
           if (full_tile)
@@ -411,7 +424,7 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
       // TMEM buffer ab is read: the contraction of tile t+2 may overwrite it
       tc_fence_before();
       fence_proxy_async_smem();
-      named_barrier_sync(2, 128);
+      named_barrier_sync(2, kMergeTmaEpi);
       if (i == 0) {
         mbar_arrive(smem_u32(&acc_empty[ab]));
         if (full_tile) {
