@@ -214,20 +214,26 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
 }
 
 // Same operation for the common case (bf16 out, d = 128, o_soft [N, H, 128]
-// bf16), streamed and warp-specialised. Warp 4 (one thread) runs a three-stage
-// TMA ring of (q, o_soft) tiles two tiles ahead of the contractions and issues
-// o_lin = q R_b into a double-buffered TMEM accumulator; warps 0-3 run the
-// epilogue (thread = row = TMEM lane) and never wait on a load. A full tile
-// of `out` is written into the q buffer of its stage (already consumed by the
-// contraction) and leaves through one TMA store; a block's ragged last tile
-// is stored row by row. Hand-offs: in_full/in_empty per stage, acc_full /
-// acc_empty per TMEM buffer.
+// bf16), streamed and warp-specialised, with separate rings for q and o_soft
+// so that neither waits on the other's release:
+//   warp 8 lane 0  issues o_lin = q R_b into a double-buffered TMEM
+//                  accumulator; each contraction's commit frees its q stage
+//   warp 8 lane 1  loads q tiles (3-stage ring), as soon as a stage is free
+//   warp 8 lane 2  loads o_soft tiles (3-stage ring)
+//   warps 0-7      epilogue: warp w reads TMEM lane quarter w % 4 and column
+//                  half w / 4 (the RMSNorm sum of squares of a row is the sum
+//                  of its halves, exchanged through shared memory); a full
+//                  tile of `out` overwrites its o_soft tile in place (each
+//                  thread rewrites the 16-byte units it read) and leaves
+//                  through one TMA store, which frees the o_soft stage once it
+//                  has read it; a block's ragged last tile is stored row by row.
 constexpr int kMergeTmaThreads = 288;          // 8 epilogue warps + the load / MMA warp
 constexpr int kMergeTmaEpi = 256;
 constexpr int kMergeTmaStages = 3;
 constexpr int kMergeTmaTiles = 14;           // 3 CTAs cover a 40-tile block
 constexpr uint32_t kMergeTmaSmemR = 0;       // 32 KB
-constexpr uint32_t kMergeTmaSmemQ = 32768;   // stage s: Q at 32 KB + 64 KB s, O_soft 32 KB after it
+constexpr uint32_t kMergeTmaSmemQ = 32768;   // q stage s at 32 KB + 32 KB s
+constexpr uint32_t kMergeTmaSmemO = 32768 + kMergeTmaStages * 32768;  // o_soft stage s
 constexpr uint32_t kMergeTmaSmemBytes = (1 + 2 * kMergeTmaStages) * 32768 + 1024;
 
 __global__ void __launch_bounds__(kMergeTmaThreads, 1)
@@ -242,7 +248,8 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
   if (ntl <= 0) return;
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t in_full[kMergeTmaStages], in_empty[kMergeTmaStages], acc_full[2], acc_empty[2];
+  __shared__ uint64_t q_full[kMergeTmaStages], q_empty[kMergeTmaStages], o_full[kMergeTmaStages],
+      o_empty[kMergeTmaStages], acc_full[2], acc_empty[2], r_ready;
   __shared__ uint32_t tmem_slot;
   __shared__ float wsm[128];
   __shared__ float ssh[2][128];  // per-row sums of squares of the two column halves
@@ -250,19 +257,22 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sR = base + kMergeTmaSmemR;
   const int i = threadIdx.x, warp = i >> 5;
-  auto sQ = [&](int st) { return base + kMergeTmaSmemQ + (uint32_t)st * 65536u; };
-  auto sO = [&](int st) { return base + kMergeTmaSmemQ + (uint32_t)st * 65536u + 32768u; };
+  auto sQ = [&](int st) { return base + kMergeTmaSmemQ + (uint32_t)st * 32768u; };
+  auto sO = [&](int st) { return base + kMergeTmaSmemO + (uint32_t)st * 32768u; };
 
   if (i == 0) {
     abort_flag = 0;
     for (int k = 0; k < kMergeTmaStages; ++k) {
-      mbar_init(smem_u32(&in_full[k]), 1);
-      mbar_init(smem_u32(&in_empty[k]), 1);
+      mbar_init(smem_u32(&q_full[k]), 1);
+      mbar_init(smem_u32(&q_empty[k]), 1);
+      mbar_init(smem_u32(&o_full[k]), 1);
+      mbar_init(smem_u32(&o_empty[k]), 1);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(smem_u32(&acc_full[k]), 1);
       mbar_init(smem_u32(&acc_empty[k]), 1);
     }
+    mbar_init(smem_u32(&r_ready), kMergeTmaEpi);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -276,31 +286,37 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
   volatile int* abort_v = &abort_flag;
 
   if (warp == 8) {
-    // ------------------------------------------------ loads and contractions
-    if (i == kMergeTmaEpi) {
-      auto load_tile = [&](int t) {
+    const int lane = i & 31;
+    if (lane == 1 || lane == 2) {
+      // -------------------------------------------------------- loaders
+      const CUtensorMap* m = lane == 1 ? &tq : &tos;
+      tma_prefetch_desc(m);
+      for (int t = 0; t < ntl; ++t) {
+        if (*abort_v) break;
         const int st = t % kMergeTmaStages;
-        const uint32_t bar = smem_u32(&in_full[st]);
-        mbar_arrive_expect_tx(bar, 65536);
+        const uint32_t ph = (uint32_t)((t / kMergeTmaStages) & 1);
+        const uint32_t empty = smem_u32(lane == 1 ? &q_empty[st] : &o_empty[st]);
+        const uint32_t full = smem_u32(lane == 1 ? &q_full[st] : &o_full[st]);
+        if (!mbar_wait(empty, ph ^ 1)) { *abort_v = 1; break; }
+        const uint32_t dst = lane == 1 ? sQ(st) : sO(st);
         const int row = q0 + (t_first + t) * kTile;
-        tma_load_3d(sQ(st), &tq, bar, 0, h, row);
-        tma_load_3d(sQ(st) + 16384, &tq, bar, 64, h, row);
-        tma_load_3d(sO(st), &tos, bar, 0, h, row);
-        tma_load_3d(sO(st) + 16384, &tos, bar, 64, h, row);
-      };
-      tma_prefetch_desc(&tq);
-      tma_prefetch_desc(&tos);
-      tma_prefetch_desc(&tout);
-      for (int t = 0; t < imin(ntl, kMergeTmaStages); ++t) load_tile(t);
+        mbar_arrive_expect_tx(full, 32768);
+        tma_load_3d(dst, m, full, 0, h, row);
+        tma_load_3d(dst + 16384, m, full, 64, h, row);
+      }
     }
-    // R_b is ready once the epilogue warps pass this barrier
-    named_barrier_sync(1, kMergeTmaThreads);
-    if (i == kMergeTmaEpi) {
+    // The three lanes run independently; none of them takes part in a named
+    // barrier, so a loader blocked on a stage never holds up the others.
+    if (lane == 0) {
+      // ----------------------------------------------------- contractions
+      tma_prefetch_desc(&tout);
       const uint32_t idO = idesc_bf16(128, 128, false, true);
+      // R_b is in shared memory once all epilogue threads have arrived
+      if (!mbar_wait(smem_u32(&r_ready), 0)) *abort_v = 1;
       for (int t = 0; t < ntl; ++t) {
         if (*abort_v) break;
         const int st = t % kMergeTmaStages, ab = t & 1;
-        if (!mbar_wait(smem_u32(&in_full[st]), (uint32_t)((t / kMergeTmaStages) & 1))) {
+        if (!mbar_wait(smem_u32(&q_full[st]), (uint32_t)((t / kMergeTmaStages) & 1))) {
           *abort_v = 1;
           break;
         }
@@ -315,30 +331,12 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
                        sdesc_sw128(sQ(st) + (uint32_t)((s >> 2) * 16384 + (s & 3) * 32), 16, 1024),
                        sdesc_sw128(sR + (uint32_t)(s * 2048), 16384, 1024), idO, s > 0 ? 1u : 0u);
         umma_commit(smem_u32(&acc_full[ab]));
-        // refill the stage of tile t-1 once its epilogue is done with it
-        const int tn = t + kMergeTmaStages - 1;
-        if (t >= 1 && tn < ntl) {
-          const int sp = (t - 1) % kMergeTmaStages;
-          if (!mbar_wait(smem_u32(&in_empty[sp]), (uint32_t)(((t - 1) / kMergeTmaStages) & 1))) {
-            *abort_v = 1;
-            break;
-          }
-          const uint32_t bar = smem_u32(&in_full[sp]);
-          mbar_arrive_expect_tx(bar, 65536);
-          const int row = q0 + (t_first + tn) * kTile;
-          tma_load_3d(sQ(sp), &tq, bar, 0, h, row);
-          tma_load_3d(sQ(sp) + 16384, &tq, bar, 64, h, row);
-          tma_load_3d(sO(sp), &tos, bar, 0, h, row);
-          tma_load_3d(sO(sp) + 16384, &tos, bar, 64, h, row);
-        }
+        umma_commit(smem_u32(&q_empty[st]));  // the q stage is free once this has run
       }
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    // 8 warps: warp w reads TMEM lane quarter w % 4 (rows 32 (w % 4) ..) and
-    // column half w / 4; the RMSNorm sum of squares of a row is the sum of
-    // its two halves, exchanged through shared memory.
     // R_b (fwd + bwd) -> bf16, MN-major 128B-swizzled: thread i converts
     // chunk i / 128 (64 value dims) of row i % 128 (key dim)
     {
@@ -361,7 +359,8 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
     }
     if (i < 128) wsm[i] = __ldg(p.rms_w + (int64_t)h * 128 + i);
     fence_proxy_async_smem();
-    named_barrier_sync(1, kMergeTmaThreads);
+    mbar_arrive(smem_u32(&r_ready));      // R_b written (async-proxy visible)
+    named_barrier_sync(2, kMergeTmaEpi);  // wsm written
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + (i & 31);   // row of the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -376,7 +375,9 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
         gsv = sigmoidf_(load_gate(p.g_s, (int64_t)row * p.H + h, p.gate_f32));
         glv = sigmoidf_(load_gate(p.g_l, (int64_t)row * p.H + h, p.gate_f32));
       }
-      const bool mine = !*abort_v && mbar_wait(smem_u32(&acc_full[ab]), (uint32_t)((t >> 1) & 1));
+      const bool mine = !*abort_v &&
+                        mbar_wait(smem_u32(&acc_full[ab]), (uint32_t)((t >> 1) & 1)) &&
+                        mbar_wait(smem_u32(&o_full[st]), (uint32_t)((t / kMergeTmaStages) & 1));
       // uniform over the 256 epilogue threads: all leave or none does
       if (!named_barrier_and(2, kMergeTmaEpi, mine)) {
         *abort_v = 1;
@@ -395,7 +396,10 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(o[c][e]), __uint_as_float(o[c][e]), ss);
       ssh[half][r] = ss;
+      // both halves' sums are written; the TMEM buffer has been read
+      tc_fence_before();
       named_barrier_sync(2, kMergeTmaEpi);
+      if (i == 0) mbar_arrive(smem_u32(&acc_empty[ab]));
       ss = ssh[0][r] + ssh[1][r];
       const float nr = glv * rsqrtf(ss * (1.f / 128.f) + p.eps);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + ((int64_t)row * p.H + h) * 128;
@@ -416,24 +420,21 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
             y4[e] = pack_bf16x2(ylo, yhi);
           }
           if (full_tile)
-            st_shared_v4(sQ(st) + off, y4[0], y4[1], y4[2], y4[3]);  // Q_t is consumed
+            st_shared_v4(sO(st) + off, y4[0], y4[1], y4[2], y4[3]);  // in place
           else if (valid)
             *reinterpret_cast<uint4*>(orow + c0) = make_uint4(y4[0], y4[1], y4[2], y4[3]);
         }
       }
-      // TMEM buffer ab is read: the contraction of tile t+2 may overwrite it
-      tc_fence_before();
       fence_proxy_async_smem();
       named_barrier_sync(2, kMergeTmaEpi);
       if (i == 0) {
-        mbar_arrive(smem_u32(&acc_empty[ab]));
         if (full_tile) {
-          tma_store_3d(&tout, sQ(st), 0, h, row0);
-          tma_store_3d(&tout, sQ(st) + 16384, 64, h, row0);
+          tma_store_3d(&tout, sO(st), 0, h, row0);
+          tma_store_3d(&tout, sO(st) + 16384, 64, h, row0);
           bulk_commit_group();
           bulk_wait_read_all();  // the stage may be refilled once the store has read it
         }
-        mbar_arrive(smem_u32(&in_empty[st]));
+        mbar_arrive(smem_u32(&o_empty[st]));
       }
     }
     if (i == 0) bulk_wait_all();
