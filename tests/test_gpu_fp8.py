@@ -70,6 +70,28 @@ def test_fp8_softmax_small(name):
     assert np.all(np.isfinite(lse.cpu().numpy()))
 
 
+def _block_size_case(bf):
+    inp = S.make_inputs_from(30 if bf == 7 else 9, [110] * 30 if bf == 7 else
+                             [37, 0, 5, 129, 64, 2, 90, 11, 40], 33 if bf == 7 else 7, 2, 128,
+                             "bf16", seed=38 + bf)
+    inp["block_frames"] = bf
+    return inp
+
+
+@pytest.mark.parametrize("name", ["max-jump", "bf1", "bf7"])
+def test_fp8_softmax_against_emulation(name):
+    # sharp attention (keys scaled by 2^(f // 2): the running max jumps by far
+    # more than 8 between tiles) and blocks of 1 and 7 frames: the kernel
+    # follows the CPU emulation of the same e4m3 method
+    from test_softmax_algorithm import _max_jump
+    inp = _max_jump() if name == "max-jump" else _block_size_case(int(name[2:]))
+    o = run_bsa_fp8(inp)[0].float().cpu().numpy()
+    for h in range(inp["H"]):
+        emu = emulate_fp8_head(inp, h)
+        assert np.all(np.isfinite(o[:, h]))
+        assert rel_l2(o[:, h], emu) <= 2e-2, (name, h)
+
+
 @pytest.mark.parametrize("name", ["pages-scale", "hi-res"])
 def test_fp8_softmax_full_sampled(name):
     inp = S.make_inputs(name)
@@ -83,7 +105,7 @@ def test_fp8_softmax_full_sampled(name):
         _check(got, ref, (name, h))
 
 
-@pytest.mark.parametrize("name", ["mid", "pages-scale"])
+@pytest.mark.parametrize("name", ["mid", "pages-scale", "hi-res"])
 def test_fp8_layer_matches_oracle(name):
     import video_diffusion_hybrid_block_b200 as V
     inp = mid_case(seed=36) if name == "mid" else S.make_inputs(name)

@@ -192,3 +192,18 @@ def test_projected_layer_full_size_sampled(name, precision):
         assert rel_l2(got, ref) <= FP8_REL_L2
         row = np.linalg.norm(got - ref, axis=1) / np.linalg.norm(ref, axis=1)
         assert row.max() <= FP8_ROW_REL_L2
+
+
+@pytest.mark.parametrize("D,precision", [(200, 0), (200, 1), (776, 1)])
+def test_projected_layer_other_widths(D, precision):
+    # output widths other than H d, including ragged 256-column tiles
+    inp = mid_case(seed=25)
+    w_o = S.make_proj_weight(inp["H"], inp["d"], D=D, seed=4)
+    y = run_proj(inp, w_o, precision)
+    ref = O.layer_proj(inp, w_o)
+    assert y.shape == (inp["N"], D)
+    if precision == 0:
+        assert rel_l2(y, ref) <= OUT_REL_L2
+        assert max_abs(y, ref) <= OUT_MAX_ABS
+    else:
+        assert rel_l2(y, ref) <= FP8_REL_L2
