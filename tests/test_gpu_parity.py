@@ -330,3 +330,48 @@ def test_split_layer_equals_layer(name):
     torch.cuda.synchronize()
     assert V.vdn_get_device_error() == 0
     assert torch.equal(got, ref)
+
+
+@pytest.mark.parametrize("name", ["mid", "d64-f32"])
+def test_layer_replays_from_a_cuda_graph(name):
+    # The layer's launches (staging, Gram + inverse, scans, packing, merged
+    # softmax kernel) are plain kernel launches on the caller's stream, so the
+    # whole call can be captured once (after a first call has done the
+    # one-time kernel-attribute set-up) and replayed; replays equal eager calls
+    # bit for bit, on new inputs copied into the captured buffers too.
+    import video_diffusion_hybrid_block_b200 as V
+    from vdn_cases import make_shape
+    inp = mid_case(seed=42) if name == "mid" else _cases(name)
+    dev = device_inputs(inp)
+    ref = run_layer(inp, dev)
+    shape = make_shape(inp)
+    ws = V.alloc_workspace(shape)
+    out = torch.empty_like(dev["q"])
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        V.vdn_hybrid_attn_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"],
+                              dev["g_s"], dev["g_l"], dev["rms_w"], out, ws, stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        V.vdn_hybrid_attn_fwd(shape, dev["q"], dev["k"], dev["v"], dev["kt"], dev["vt"],
+                              dev["g_s"], dev["g_l"], dev["rms_w"], out, ws)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert V.vdn_get_device_error() == 0
+        assert torch.equal(out, ref)
+    # new inputs through the same captured buffers
+    inp2 = mid_case(seed=43) if name == "mid" else _cases(name)
+    if name != "mid":
+        inp2 = dict(inp2)
+        inp2["q"] = inp2["q"] * 0.5
+    dev2 = device_inputs(inp2)
+    for key in ("q", "k", "v", "kt", "vt", "g_s", "g_l"):
+        dev[key].copy_(dev2[key])
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, run_layer(inp2, dev2))
