@@ -609,7 +609,10 @@ def run_cuda(args) -> None:
 
     # ---- every workload; the headline's report reuses its layer time
     reports = {}
-    names = [args.workload] if args.workloads == "none" else WORKLOADS
+    # the extra reports run at N = 1; at N > 1 (replicas) only the headline
+    # workload is reported, which keeps the multi-GPU run short
+    full_report = args.workloads == "all" or (args.workloads == "auto" and world == 1)
+    names = WORKLOADS if full_report else [args.workload]
     for name in names:
         ww = w if name == args.workload else Workload(name, V, torch)
         reports[name] = workload_report(V, torch, ww, stream, args.steps, args.warmup, peaks,
@@ -619,7 +622,7 @@ def run_cuda(args) -> None:
             del ww
             torch.cuda.empty_cache()
     proj = fp8 = None
-    if not args.no_projections and w.inp["d"] == 128 and w.inp["dtype"] == "bf16":
+    if full_report and not args.no_projections and w.inp["d"] == 128 and w.inp["dtype"] == "bf16":
         proj = projection_report(V, torch, w, stream, args.steps, peaks)
         fp8 = fp8_report(V, torch, w, stream, args.steps, peaks)
     head = reports[args.workload]
@@ -829,8 +832,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-projections", action="store_true",
                     help="skip the per-branch output projection measurements")
-    ap.add_argument("--workloads", default="all", choices=["all", "none"],
-                    help="also report every workload (default) or only the headline one")
+    ap.add_argument("--workloads", default="auto", choices=["auto", "all", "none"],
+                    help="also report every workload, the projections and the e4m3 figures "
+                         "(auto: on one GPU only), or only the headline workload")
     ap.add_argument("--profile", choices=["layer", "bsa", "vda", "merge", "proj", "proj8", "bsa8"],
                     help="only run launches of one entry point (for ncu captures)")
     ap.add_argument("--workload", default=HEADLINE,
