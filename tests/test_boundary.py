@@ -255,3 +255,14 @@ def test_split_layer_checks(lib):
     assert lib.vdn_bsa_merge_fwd(s.ref, *args, None, FAKE, FAKE, need, 0) == B.VDN_ERR_INVALID_ARG
     assert lib.vdn_bsa_merge_fwd(s.ref, *args, FAKE, FAKE, FAKE, need - 1, 0) == \
         B.VDN_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_index_limit(lib):
+    # N * H * 128 must stay below 2^31; one head more than the largest
+    # accepted count is rejected before any launch
+    off = S.frame_offsets([256] * 16)
+    ok, bad = shape(off=off, H=4095), shape(off=off, H=4096)
+    assert V.vdn_workspace_bytes(ok) > 0
+    assert V.vdn_workspace_bytes(bad) == 0
+    assert lib.vdn_hybrid_attn_fwd(bad.ref, *([FAKE] * 9), FAKE, 1 << 40, 0) == \
+        B.VDN_ERR_UNSUPPORTED

@@ -21,6 +21,8 @@ q, k, v, kt, vt, g_s, g_l.
 * gate logits g_s, g_l ~ N(0, 1) with shape [N, H]; RMSNorm weight = 1 [H, d].
 * bf16 workloads round every float input to bf16 (round to nearest even);
   the returned float32 arrays then hold exactly the bf16 values.
+* make_inputs_device: the same distributions drawn on the device with
+  torch's Philox generator (for shapes too large for the host).
 * output-projection weights (make_proj_weight): w_o [D, 2 H d] ~
   N(0, 1) / sqrt(2 H d), default_rng(seed + 1000), bf16.
 """
@@ -135,6 +137,37 @@ def make_proj_weight(H: int, d: int, D: int | None = None, seed: int = 0) -> np.
     rng = np.random.default_rng(seed + 1000)
     w = rng.standard_normal((D, 2 * H * d), dtype=np.float32) / np.float32(np.sqrt(2 * H * d))
     return bf16_round(w)
+
+
+def make_inputs_device(F, sizes, T, H, d, seed=0, device="cuda"):
+    """Inputs too large to draw on the host, drawn on the device: torch's
+    Philox generator seeded with `seed`, float32 draws in the order q, k, v,
+    kt, vt, g_s, g_l (N(0, 1); k and kt L2-normalised), rounded to bf16.
+    Returns torch tensors plus the frame offsets and the layer constants."""
+    import torch
+    sizes = np.asarray(sizes, dtype=np.int64)
+    off = frame_offsets(sizes)
+    N = int(off[-1])
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    out = {}
+    for key, shape in (("q", (N, H, d)), ("k", (N, H, d)), ("v", (N, H, d)), ("kt", (T, H, d)),
+                       ("vt", (T, H, d)), ("g_s", (N, H)), ("g_l", (N, H))):
+        x = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        # draw in row chunks so no full-size float32 copy is ever held
+        rows = max(1, (1 << 26) // max(1, int(np.prod(shape[1:]))))
+        for r0 in range(0, shape[0], rows):
+            r1 = min(shape[0], r0 + rows)
+            y = torch.randn((r1 - r0,) + shape[1:], generator=g, device=device,
+                            dtype=torch.float32)
+            if key in ("k", "kt"):
+                y = y / torch.clamp(y.norm(dim=-1, keepdim=True), min=1e-12)
+            x[r0:r1] = y.to(torch.bfloat16)
+        out[key] = x
+    out["rms_w"] = torch.ones((H, d), dtype=torch.float32, device=device)
+    out.update(off=off, F=F, T=T, H=H, d=d, N=N, dtype="bf16", block_frames=BLOCK_FRAMES,
+               lam=LAMBDA, eps=RMS_EPS)
+    return out
 
 
 def make_inputs(name: str, seed: int = 0) -> dict:
