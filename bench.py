@@ -167,31 +167,84 @@ def recorded_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms (read only)."""
+    """SM clock and clock-event reasons of the GPU this process runs on, read
+    (never set) while a timed region runs. NVML is polled every 5 ms from a
+    thread; without NVML, nvidia-smi samples at its 200 ms floor. The device
+    is found by its UUID, so the samples come from this process's GPU
+    whatever CUDA_VISIBLE_DEVICES maps. Samples flagged GPU-idle are left
+    out of the median (a region can hold idle pauses)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # clock-event reason bits of NVML's public header
+    IDLE = 0x1
+    REASONS = (("hw_slowdown", 0x8 | 0x80), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+    PERIOD_S = 0.005
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, device: int):
+        self.device = device
+        self.samples = []  # (sm_mhz, sm_max_mhz, reason bits)
         self.proc = None
         self.path = None
+        self.thread = None
+        self.stop = None
+        self.source = None
+
+    def _uuid(self):
+        try:
+            import torch
+            return "GPU-" + str(torch.cuda.get_device_properties(self.device).uuid)
+        except Exception:
+            return None
+
+    def _nvml_poll(self, nv, h, ready):
+        clk_sm = nv.NVML_CLOCK_SM
+        reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, clk_sm)
+        while True:
+            self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, clk_sm)), float(smax),
+                                 int(reasons(h))))
+            ready.set()
+            if self.stop.wait(self.PERIOD_S):
+                return
 
     def __enter__(self):
+        import threading
+        uuid = self._uuid()
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByUUID(uuid) if uuid else \
+                nv.nvmlDeviceGetHandleByIndex(self.device)
+            self.stop, ready = threading.Event(), threading.Event()
+            self.thread = threading.Thread(target=self._nvml_poll, args=(nv, h, ready),
+                                           daemon=True)
+            self.thread.start()
+            ready.wait(1.0)
+            self.source = f"nvml every {self.PERIOD_S * 1e3:.0f} ms"
+            return self
+        except Exception:
+            self.thread = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={uuid or self.device}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi every 200 ms"
         except OSError:
             self.proc = None
         time.sleep(0.3)
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -199,24 +252,40 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
+    def _read_smi(self):
+        if not (self.path and os.path.exists(self.path)):
+            return
+        names = dict(self.REASONS)
+        with open(self.path) as fh:
+            for line in fh:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9 or not p[1].replace(".", "").isdigit():
+                    continue
+                bits = 0
+                for i, n in enumerate(("hw_slowdown", "hw_thermal_slowdown",
+                                       "sw_thermal_slowdown", "sw_power_cap")):
+                    if p[5 + i] == "Active":
+                        bits |= names[n]
+                smax = float(p[2]) if p[2].replace(".", "").isdigit() else 0.0
+                self.samples.append((float(p[1]), smax, bits))
+        os.unlink(self.path)
+        self.path = None
+
     def summary(self) -> dict:
-        rows = []
-        if self.path and os.path.exists(self.path):
-            with open(self.path) as fh:
-                for line in fh:
-                    parts = [p.strip() for p in line.split(",")]
-                    if len(parts) >= 9:
-                        rows.append(parts)
-            os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
-                "samples": len(rows)}
+        self._read_smi()
+        return summarize_clock_samples(self.samples, self.IDLE, self.REASONS, self.source)
+
+
+def summarize_clock_samples(samples, idle_bit: int, reasons, source) -> dict:
+    """Median SM clock over the busy samples, the max clock and every
+    slowdown reason seen in any busy sample."""
+    if not samples:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    busy = [s for s in samples if not s[2] & idle_bit] or samples
+    seen = sorted({n for _, _, b in busy for n, m in reasons if b & m})
+    return {"sm_mhz": statistics.median(s[0] for s in busy),
+            "sm_max_mhz": max(s[1] for s in samples), "reasons": seen,
+            "samples": len(busy), "idle_samples": len(samples) - len(busy), "source": source}
 
 
 def max_over_ranks(dist, x: float, device) -> float:

@@ -110,3 +110,19 @@ def test_config_is_shared_by_both_arms():
     a = bench.config_of("tiny", inp, fl, 1)
     assert set(a) >= {"workload", "F", "N", "T", "H", "d", "parallelism", "l2"}
     assert "fit in the 126 MB L2" in a["l2"]
+
+
+def test_clock_summary_drops_idle_samples_and_maps_reasons():
+    """Idle samples stay out of the median; every slowdown bit seen in a busy
+    sample is named (hardware power brake counts as hw_slowdown)."""
+    C = bench.ClockSampler
+    s = [(345.0, 1965.0, C.IDLE), (1965.0, 1965.0, 0x4), (1950.0, 1965.0, 0x4),
+         (1800.0, 1965.0, 0x80), (300.0, 1965.0, C.IDLE | 0x20)]
+    r = bench.summarize_clock_samples(s, C.IDLE, C.REASONS, "test")
+    assert r["sm_mhz"] == 1950.0 and r["sm_max_mhz"] == 1965.0
+    assert r["samples"] == 3 and r["idle_samples"] == 2
+    assert r["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert bench.summarize_clock_samples([], C.IDLE, C.REASONS, "test")["reasons"] == ["no samples"]
+    # all samples idle: the median falls back to all of them
+    r = bench.summarize_clock_samples(s[:1], C.IDLE, C.REASONS, "test")
+    assert r["sm_mhz"] == 345.0

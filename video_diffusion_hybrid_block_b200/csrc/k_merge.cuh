@@ -220,13 +220,17 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
 //                  accumulator; each contraction's commit frees its q stage
 //   warp 8 lane 1  loads q tiles (3-stage ring), as soon as a stage is free
 //   warp 8 lane 2  loads o_soft tiles (3-stage ring)
+//   warp 8 lane 3  stores: once all epilogue threads have staged a full tile
+//                  it sends it with one TMA store, waits until the store has
+//                  read the stage and frees it for the o_soft loader
 //   warps 0-7      epilogue: warp w reads TMEM lane quarter w % 4 and column
 //                  half w / 4 (the RMSNorm sum of squares of a row is the sum
 //                  of its halves, exchanged through shared memory); a full
 //                  tile of `out` overwrites its o_soft tile in place (each
-//                  thread rewrites the 16-byte units it read) and leaves
-//                  through one TMA store, which frees the o_soft stage once it
-//                  has read it; a block's ragged last tile is stored row by row.
+//                  thread rewrites the 16-byte units it read) and is handed
+//                  to the store lane, so the epilogue moves on to the next
+//                  tile without waiting for the store; a block's ragged last
+//                  tile is stored row by row.
 constexpr int kMergeTmaThreads = 288;          // 8 epilogue warps + the load / MMA warp
 constexpr int kMergeTmaEpi = 256;
 constexpr int kMergeTmaStages = 3;
@@ -249,7 +253,7 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full[kMergeTmaStages], q_empty[kMergeTmaStages], o_full[kMergeTmaStages],
-      o_empty[kMergeTmaStages], acc_full[2], acc_empty[2], r_ready;
+      o_empty[kMergeTmaStages], o_staged[kMergeTmaStages], acc_full[2], acc_empty[2], r_ready;
   __shared__ uint32_t tmem_slot;
   __shared__ float wsm[128];
   __shared__ float ssh[2][128];  // per-row sums of squares of the two column halves
@@ -267,6 +271,7 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
       mbar_init(smem_u32(&q_empty[k]), 1);
       mbar_init(smem_u32(&o_full[k]), 1);
       mbar_init(smem_u32(&o_empty[k]), 1);
+      mbar_init(smem_u32(&o_staged[k]), kMergeTmaEpi);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(smem_u32(&acc_full[k]), 1);
@@ -305,11 +310,31 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
         tma_load_3d(dst + 16384, m, full, 64, h, row);
       }
     }
-    // The three lanes run independently; none of them takes part in a named
-    // barrier, so a loader blocked on a stage never holds up the others.
+    if (lane == 3) {
+      // ------------------------------------------------------------ stores
+      tma_prefetch_desc(&tout);
+      for (int t = 0; t < ntl; ++t) {
+        if (*abort_v) break;
+        const int st = t % kMergeTmaStages;
+        if (!mbar_wait(smem_u32(&o_staged[st]), (uint32_t)((t / kMergeTmaStages) & 1))) {
+          *abort_v = 1;
+          break;
+        }
+        const int row0 = q0 + (t_first + t) * kTile;
+        if (row0 + kTile <= q1) {
+          tma_store_3d(&tout, sO(st), 0, h, row0);
+          tma_store_3d(&tout, sO(st) + 16384, 64, h, row0);
+          bulk_commit_group();
+          bulk_wait_read_all();  // the stage may be refilled once the store has read it
+        }
+        mbar_arrive(smem_u32(&o_empty[st]));
+      }
+      bulk_wait_all();
+    }
+    // The four lanes run independently; none of them takes part in a named
+    // barrier, so a lane blocked on a stage never holds up the others.
     if (lane == 0) {
       // ----------------------------------------------------- contractions
-      tma_prefetch_desc(&tout);
       const uint32_t idO = idesc_bf16(128, 128, false, true);
       // R_b is in shared memory once all epilogue threads have arrived
       if (!mbar_wait(smem_u32(&r_ready), 0)) *abort_v = 1;
@@ -425,19 +450,11 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
             *reinterpret_cast<uint4*>(orow + c0) = make_uint4(y4[0], y4[1], y4[2], y4[3]);
         }
       }
+      // this thread's part of the tile is staged (or, for a ragged tile,
+      // its reads of the o_soft stage are done)
       fence_proxy_async_smem();
-      named_barrier_sync(2, kMergeTmaEpi);
-      if (i == 0) {
-        if (full_tile) {
-          tma_store_3d(&tout, sO(st), 0, h, row0);
-          tma_store_3d(&tout, sO(st) + 16384, 64, h, row0);
-          bulk_commit_group();
-          bulk_wait_read_all();  // the stage may be refilled once the store has read it
-        }
-        mbar_arrive(smem_u32(&o_empty[st]));
-      }
+      mbar_arrive(smem_u32(&o_staged[st]));
     }
-    if (i == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
