@@ -389,16 +389,30 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + (i & 31);   // row of the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    // gate logits one tile ahead, kept as raw bits until the next tile uses
+    // them: a conversion right after the load would stall the warp for the
+    // load's whole latency
+    auto gate_bits = [&](const void* g, int row) -> uint32_t {
+      if (row >= q1) return 0u;
+      const int64_t gi = (int64_t)row * p.H + h;
+      return p.gate_f32 ? __float_as_uint(__ldg(reinterpret_cast<const float*>(g) + gi))
+                        : (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(g) + gi);
+    };
+    auto gate_val = [&](uint32_t bits) -> float {
+      return sigmoidf_(p.gate_f32 ? __uint_as_float(bits) : __uint_as_float(bits << 16));
+    };
+    uint32_t gs_next = gate_bits(p.g_s, q0 + t_first * kTile + r);
+    uint32_t gl_next = gate_bits(p.g_l, q0 + t_first * kTile + r);
     for (int t = 0; t < ntl; ++t) {
       const int st = t % kMergeTmaStages, ab = t & 1;
       const int row0 = q0 + (t_first + t) * kTile;
       const int row = row0 + r;
       const bool valid = row < q1;
       const bool full_tile = row0 + kTile <= q1;
-      float gsv = 0.f, glv = 0.f;
-      if (valid) {
-        gsv = sigmoidf_(load_gate(p.g_s, (int64_t)row * p.H + h, p.gate_f32));
-        glv = sigmoidf_(load_gate(p.g_l, (int64_t)row * p.H + h, p.gate_f32));
+      const uint32_t gs_bits = gs_next, gl_bits = gl_next;
+      if (t + 1 < ntl) {
+        gs_next = gate_bits(p.g_s, row + kTile);
+        gl_next = gate_bits(p.g_l, row + kTile);
       }
       const bool mine = !*abort_v &&
                         mbar_wait(smem_u32(&acc_full[ab]), (uint32_t)((t >> 1) & 1)) &&
@@ -426,7 +440,8 @@ __global__ void __launch_bounds__(kMergeTmaThreads, 1)
       named_barrier_sync(2, kMergeTmaEpi);
       if (i == 0) mbar_arrive(smem_u32(&acc_empty[ab]));
       ss = ssh[0][r] + ssh[1][r];
-      const float nr = glv * rsqrtf(ss * (1.f / 128.f) + p.eps);
+      const float gsv = valid ? gate_val(gs_bits) : 0.f;
+      const float nr = (valid ? gate_val(gl_bits) : 0.f) * rsqrtf(ss * (1.f / 128.f) + p.eps);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + ((int64_t)row * p.H + h) * 128;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
