@@ -266,6 +266,35 @@ def test_gate_merge_entry_matches_layer(d):
         assert max_abs(got[:, h], oref) <= OUT_MAX_ABS, h
 
 
+@pytest.mark.parametrize("rows", [(100, 1792), (1920, 3650)])
+def test_gate_merge_tile_counts(rows):
+    # the streamed merge kernel at block sizes around its ring and CTA
+    # boundaries (3 stages, 14 tiles per CTA): one ragged tile, exactly 14
+    # full tiles, 14 + 1, and 14 + 14 + one ragged tile
+    import video_diffusion_hybrid_block_b200 as V
+    from vdn_cases import make_shape
+    sizes = []
+    for n in rows:
+        base = n // 5
+        sizes += [base] * 4 + [n - 4 * base]
+    inp = S.make_inputs_from(len(sizes), sizes, 16, 2, 128, "bf16", seed=41)
+    dev = device_inputs(inp)
+    o, _ = run_bsa(inp, dev)
+    R, _, _, _ = run_scan(inp, dev, per_frame=False)
+    shape = make_shape(inp)
+    ws = V.alloc_workspace(shape)
+    out = torch.empty_like(dev["q"])
+    V.vdn_gate_merge(shape, dev["q"], R, o, dev["g_s"], dev["g_l"], dev["rms_w"], out, ws)
+    torch.cuda.synchronize()
+    assert V.vdn_get_device_error() == 0
+    got = out.float().cpu().numpy()
+    assert rel_l2(got, run_layer(inp, dev).float().cpu().numpy()) <= 1e-2
+    for h in range(inp["H"]):
+        oref = O.layer_head(inp, h)["out"]
+        assert rel_l2(got[:, h], oref) <= OUT_REL_L2, h
+        assert max_abs(got[:, h], oref) <= OUT_MAX_ABS, h
+
+
 def test_profile_entry_matches_layer():
     # the measurement helper runs the same launches: identical output, and a
     # positive time for every kernel group the bf16 d = 128 layer launches
