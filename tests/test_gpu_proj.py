@@ -108,7 +108,7 @@ def test_linear_bf16_matches_fp64(M, K, D):
     assert max_abs(got, ref) <= 1e-2 * np.abs(ref).max() + 1e-3
 
 
-@pytest.mark.parametrize("rows,K", [(37, 48), (1000, 6144), (4, 16)])
+@pytest.mark.parametrize("rows,K", [(37, 48), (1000, 6144), (5, 6160), (4, 16)])
 def test_quantize_rows_bit_exact(rows, K):
     V = _V()
     rng = np.random.default_rng(rows)

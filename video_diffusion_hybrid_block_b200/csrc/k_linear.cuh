@@ -232,43 +232,74 @@ __global__ void __launch_bounds__(kLinThreads, 1)
 
 // Per-row e4m3 quantisation of a bf16 matrix [rows, K] (K % 8 == 0), one warp
 // per row: scales[row] = amax / 448, codes = e4m3(x * (448 / amax)).
+// Rows of up to kQuantRegUnits x 32 16-byte units (K <= 6144) stay in
+// registers between the amax and the code pass, so each row is read from
+// memory once and all of a lane's loads are in flight together; longer rows
+// are read twice.
+constexpr int kQuantRegUnits = 24;
+
+__device__ __forceinline__ float amax_bf16x8(uint4 u) {
+  const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+  float m = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf_lo(w4[e])), fabsf(bf_hi(w4[e]))));
+  return m;
+}
+
+// 8 bf16 values times inv -> 8 e4m3 codes, in memory order
+__device__ __forceinline__ uint2 codes_bf16x8(uint4 u, float inv) {
+  const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+  uint32_t packed[2];
+#pragma unroll
+  for (int e = 0; e < 4; e += 2) {
+    uint16_t lo, hi;
+    // the first source lands in the upper byte: (x1, x0) puts x0 first in memory
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+        : "=h"(lo)
+        : "f"(__fmul_rn(bf_hi(w4[e]), inv)), "f"(__fmul_rn(bf_lo(w4[e]), inv)));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+        : "=h"(hi)
+        : "f"(__fmul_rn(bf_hi(w4[e + 1]), inv)), "f"(__fmul_rn(bf_lo(w4[e + 1]), inv)));
+    packed[e >> 1] = (uint32_t)lo | ((uint32_t)hi << 16);
+  }
+  return make_uint2(packed[0], packed[1]);
+}
+
 __global__ void k_quant_rows_e4m3(const __nv_bfloat16* __restrict__ x, int64_t rows, int K,
                                   uint8_t* __restrict__ codes, float* __restrict__ scales) {
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   const uint4* src = reinterpret_cast<const uint4*>(x + row * K);
+  uint2* dst = reinterpret_cast<uint2*>(codes + row * K);
   const int nv = K >> 3;
   float amax = 0.f;
-  for (int i = lane; i < nv; i += 32) {
-    const uint4 u = __ldg(src + i);
-    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+  if (nv <= kQuantRegUnits * 32) {
+    uint4 xr[kQuantRegUnits];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf_lo(w4[e])), fabsf(bf_hi(w4[e]))));
+    for (int u = 0; u < kQuantRegUnits; ++u) {
+      const int i = lane + 32 * u;
+      xr[u] = i < nv ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantRegUnits; ++u) amax = fmaxf(amax, amax_bf16x8(xr[u]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+    if (lane == 0) scales[row] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+#pragma unroll
+    for (int u = 0; u < kQuantRegUnits; ++u) {
+      const int i = lane + 32 * u;
+      if (i < nv) dst[i] = codes_bf16x8(xr[u], inv);
+    }
+    return;
   }
+  for (int i = lane; i < nv; i += 32) amax = fmaxf(amax, amax_bf16x8(__ldg(src + i)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
   if (lane == 0) scales[row] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-  uint2* dst = reinterpret_cast<uint2*>(codes + row * K);
-  for (int i = lane; i < nv; i += 32) {
-    const uint4 u = __ldg(src + i);
-    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-    uint32_t packed[2];
-#pragma unroll
-    for (int e = 0; e < 4; e += 2) {
-      uint16_t lo, hi;
-      // the first source lands in the upper byte: (x1, x0) puts x0 first in memory
-      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-          : "=h"(lo)
-          : "f"(__fmul_rn(bf_hi(w4[e]), inv)), "f"(__fmul_rn(bf_lo(w4[e]), inv)));
-      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-          : "=h"(hi)
-          : "f"(__fmul_rn(bf_hi(w4[e + 1]), inv)), "f"(__fmul_rn(bf_lo(w4[e + 1]), inv)));
-      packed[e >> 1] = (uint32_t)lo | ((uint32_t)hi << 16);
-    }
-    dst[i] = make_uint2(packed[0], packed[1]);
-  }
+  for (int i = lane; i < nv; i += 32) dst[i] = codes_bf16x8(__ldg(src + i), inv);
 }
 
 }  // namespace vdn
