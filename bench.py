@@ -277,14 +277,15 @@ class ClockSampler:
 
 
 def summarize_clock_samples(samples, idle_bit: int, reasons, source) -> dict:
-    """Median SM clock over the busy samples, the max clock and every
-    slowdown reason seen in any busy sample."""
+    """Median, mean and lowest SM clock over the busy samples, the max clock
+    and every slowdown reason seen in any busy sample."""
     if not samples:
         return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
     busy = [s for s in samples if not s[2] & idle_bit] or samples
     seen = sorted({n for _, _, b in busy for n, m in reasons if b & m})
-    return {"sm_mhz": statistics.median(s[0] for s in busy),
-            "sm_max_mhz": max(s[1] for s in samples), "reasons": seen,
+    clk = [s[0] for s in busy]
+    return {"sm_mhz": statistics.median(clk), "sm_mhz_mean": round(statistics.fmean(clk), 1),
+            "sm_mhz_min": min(clk), "sm_max_mhz": max(s[1] for s in samples), "reasons": seen,
             "samples": len(busy), "idle_samples": len(samples) - len(busy), "source": source}
 
 
@@ -435,6 +436,7 @@ def workload_report(V, torch, w: Workload, stream, steps: int, warmup: int, peak
         rep["hbm"] = hbm
     c = clk.summary()
     rep["sm_mhz"] = c["sm_mhz"]
+    rep["sm_mhz_mean"] = c.get("sm_mhz_mean")
     rep["clock_reasons"] = c["reasons"]
     torch.cuda.synchronize()
     rc = V.vdn_get_device_error()

@@ -120,6 +120,7 @@ def test_clock_summary_drops_idle_samples_and_maps_reasons():
          (1800.0, 1965.0, 0x80), (300.0, 1965.0, C.IDLE | 0x20)]
     r = bench.summarize_clock_samples(s, C.IDLE, C.REASONS, "test")
     assert r["sm_mhz"] == 1950.0 and r["sm_max_mhz"] == 1965.0
+    assert r["sm_mhz_min"] == 1800.0 and r["sm_mhz_mean"] == 1905.0
     assert r["samples"] == 3 and r["idle_samples"] == 2
     assert r["reasons"] == ["hw_slowdown", "sw_power_cap"]
     assert bench.summarize_clock_samples([], C.IDLE, C.REASONS, "test")["reasons"] == ["no samples"]
