@@ -266,3 +266,56 @@ def test_index_limit(lib):
     assert V.vdn_workspace_bytes(bad) == 0
     assert lib.vdn_hybrid_attn_fwd(bad.ref, *([FAKE] * 9), FAKE, 1 << 40, 0) == \
         B.VDN_ERR_UNSUPPORTED
+
+
+def test_fp8_entry_checks(lib):
+    # e4m3 softmax branch and layer: bf16 with d = 128 only; a workspace
+    # sized for the bf16 layer is too small for the e4m3 codes
+    s = shape()
+    need = V.vdn_workspace_bytes(s)
+    need8 = lib.vdn_fp8_workspace_bytes(s.ref)
+    assert need8 > need
+    for bad in (shape(dtype=1), shape(d=64)):
+        assert lib.vdn_fp8_workspace_bytes(bad.ref) == 0
+        assert lib.vdn_bsa_fwd_fp8(bad.ref, *([FAKE] * 7), FAKE, 1 << 40, 0) == \
+            B.VDN_ERR_UNSUPPORTED
+        assert lib.vdn_hybrid_attn_fwd_fp8(bad.ref, *([FAKE] * 9), FAKE, 1 << 40, 0) == \
+            B.VDN_ERR_UNSUPPORTED
+    bsa = [FAKE] * 7  # q, k, v, kt, vt, o_soft, lse
+    for i in (0, 1, 2, 5):
+        p = list(bsa)
+        p[i] = 0
+        assert lib.vdn_bsa_fwd_fp8(s.ref, *p, FAKE, need8, 0) == B.VDN_ERR_INVALID_ARG, i
+        p[i] = FAKE_MIS
+        assert lib.vdn_bsa_fwd_fp8(s.ref, *p, FAKE, need8, 0) == B.VDN_ERR_MISALIGNED, i
+    p = list(bsa)
+    p[6] = FAKE_MIS
+    assert lib.vdn_bsa_fwd_fp8(s.ref, *p, FAKE, need8, 0) == B.VDN_ERR_MISALIGNED
+    for ws, n in ((FAKE, need8 - 1), (FAKE, need), (None, need8)):
+        assert lib.vdn_bsa_fwd_fp8(s.ref, *bsa, ws, n, 0) == B.VDN_ERR_WORKSPACE_TOO_SMALL
+        assert lib.vdn_hybrid_attn_fwd_fp8(s.ref, *([FAKE] * 9), ws, n, 0) == \
+            B.VDN_ERR_WORKSPACE_TOO_SMALL
+    assert lib.vdn_bsa_fwd_fp8(s.ref, *bsa, FAKE_MIS, need8, 0) == B.VDN_ERR_MISALIGNED
+    for i in range(9):
+        p = [FAKE] * 9
+        p[i] = 0
+        assert lib.vdn_hybrid_attn_fwd_fp8(s.ref, *p, FAKE, need8, 0) == \
+            B.VDN_ERR_INVALID_ARG, i
+
+
+def test_profile_entry_checks(lib):
+    # iteration count 1..256 and a result array are required
+    s = shape()
+    need = V.vdn_workspace_bytes(s)
+    ms = (ctypes.c_float * 5)()
+    for iters in (0, -1, 257):
+        assert lib.vdn_hybrid_attn_fwd_profile(s.ref, *([FAKE] * 9), FAKE, need, 0, iters,
+                                               ms) == B.VDN_ERR_INVALID_ARG, iters
+    assert lib.vdn_hybrid_attn_fwd_profile(s.ref, *([FAKE] * 9), FAKE, need, 0, 4, None) == \
+        B.VDN_ERR_INVALID_ARG
+    assert lib.vdn_hybrid_attn_fwd_profile(s.ref, *([FAKE] * 9), FAKE, need - 1, 0, 4, ms) == \
+        B.VDN_ERR_WORKSPACE_TOO_SMALL
+    p = [FAKE] * 9
+    p[0] = 0
+    assert lib.vdn_hybrid_attn_fwd_profile(s.ref, *p, FAKE, need, 0, 4, ms) == \
+        B.VDN_ERR_INVALID_ARG
