@@ -648,25 +648,38 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
 // R_b = Rfwd + Rbwd (fp32, padded 128 x 128) -> bf16 tile image laid out
 // exactly as the merge variant's shared-memory B operand (128B-swizzled,
 // MN-major: row k of 128 B per 64 value dims, two 16 KB chunks), so the CTA
-// fetches it with one bulk copy. One CTA per (block, head), thread = row.
+// fetches it with one bulk copy. Grid (block x head, kPackSplit row groups),
+// 128 threads; a unit is 8 consecutive values of one row (32 B of each
+// input, one 16-byte unit of the image), consecutive threads take
+// consecutive units, so each warp reads whole 512-byte rows; all of a
+// thread's loads are issued before its stores.
+constexpr int kPackSplit = 4;
+constexpr int kPackUnits = 128 * 16 / kPackSplit / 128;  // units per thread
+
 __global__ void k_pack_read_states(const float* __restrict__ ra, const float* __restrict__ rb,
                                    uint8_t* __restrict__ img) {
   const int64_t bh = blockIdx.x;
-  const int i = threadIdx.x;
-  const float4* a = reinterpret_cast<const float4*>(ra + (bh * 128 + i) * 128);
-  const float4* c4 = reinterpret_cast<const float4*>(rb + (bh * 128 + i) * 128);
+  const float4* a = reinterpret_cast<const float4*>(ra + bh * 128 * 128);
+  const float4* c4 = reinterpret_cast<const float4*>(rb + bh * 128 * 128);
   uint8_t* dst = img + bh * kRImageBytes;
+  const int u0 = (int)blockIdx.y * (128 * 16 / kPackSplit) + (int)threadIdx.x;
+  float4 x[kPackUnits][2], y[kPackUnits][2];
 #pragma unroll
-  for (int ch = 0; ch < 2; ++ch) {
+  for (int j = 0; j < kPackUnits; ++j) {
+    const int u = u0 + j * 128;  // row u / 16, values 8 (u % 16) ..
+    x[j][0] = __ldg(a + 2 * u);
+    x[j][1] = __ldg(a + 2 * u + 1);
+    y[j][0] = __ldg(c4 + 2 * u);
+    y[j][1] = __ldg(c4 + 2 * u + 1);
+  }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int q = ch * 16 + u * 2;
-      const float4 x0 = __ldg(a + q), x1 = __ldg(a + q + 1);
-      const float4 y0 = __ldg(c4 + q), y1 = __ldg(c4 + q + 1);
-      *reinterpret_cast<uint4*>(dst + ch * 16384 + sw128_off((uint32_t)i, (uint32_t)u)) =
-          make_uint4(pack_bf16x2(x0.x + y0.x, x0.y + y0.y), pack_bf16x2(x0.z + y0.z, x0.w + y0.w),
-                     pack_bf16x2(x1.x + y1.x, x1.y + y1.y), pack_bf16x2(x1.z + y1.z, x1.w + y1.w));
-    }
+  for (int j = 0; j < kPackUnits; ++j) {
+    const int u = u0 + j * 128;
+    const int row = u >> 4, c8 = u & 15;
+    const float4 p0 = x[j][0], p1 = x[j][1], q0 = y[j][0], q1 = y[j][1];
+    *reinterpret_cast<uint4*>(dst + (c8 >> 3) * 16384 + sw128_off((uint32_t)row, (uint32_t)(c8 & 7))) =
+        make_uint4(pack_bf16x2(p0.x + q0.x, p0.y + q0.y), pack_bf16x2(p0.z + q0.z, p0.w + q0.w),
+                   pack_bf16x2(p1.x + q1.x, p1.y + q1.y), pack_bf16x2(p1.z + q1.z, p1.w + q1.w));
   }
 }
 

@@ -665,8 +665,8 @@ int layer_launches(const Plan& P, const void* q, const void* k, const void* v, c
   if (rc != VDN_OK) return rc;
   if (ev != nullptr) cudaEventRecord(ev[3], st);
   const float* R = reinterpret_cast<const float*>(ws + P.o_R);
-  k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
-                                                 ws + P.o_Rimg);
+  k_pack_read_states<<<dim3(P.nb * P.H, kPackSplit), 128, 0, st>>>(
+      R, R + (size_t)P.nb * P.H * 128 * 128, ws + P.o_Rimg);
   if (ev != nullptr) cudaEventRecord(ev[4], st);
   MergeArgs m{g_s, g_l, rms_w, out, branches};
   rc = launch_bsa(P, a, ws, nullptr, 0, kDPad, nullptr, st, &m);
@@ -879,8 +879,8 @@ int vdn_hybrid_attn_fwd_fp8(const vdn_shape_t* shape, const void* q, const void*
   if (rc == VDN_OK) rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr);
   if (rc == VDN_OK) {
     const float* R = reinterpret_cast<const float*>(ws + P.o_R);
-    k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
-                                                   ws + P.o_Rimg);
+    k_pack_read_states<<<dim3(P.nb * P.H, kPackSplit), 128, 0, st>>>(
+        R, R + (size_t)P.nb * P.H * 128 * 128, ws + P.o_Rimg);
     MergeArgs m{g_s, g_l, rms_w, out};
     rc = launch_bsa_fp8(P, Q, ws, nullptr, 0, nullptr, st, &m, q);
   }
@@ -910,8 +910,8 @@ int vdn_vda_read_images(const vdn_shape_t* shape, const void* k, const void* v, 
   rc = launch_vda(P, a, ws, st, nullptr, nullptr, nullptr);
   if (rc != VDN_OK) return finish(rc);
   const float* R = reinterpret_cast<const float*>(ws + P.o_R);
-  k_pack_read_states<<<P.nb * P.H, 128, 0, st>>>(R, R + (size_t)P.nb * P.H * 128 * 128,
-                                                 static_cast<uint8_t*>(rimg));
+  k_pack_read_states<<<dim3(P.nb * P.H, kPackSplit), 128, 0, st>>>(
+      R, R + (size_t)P.nb * P.H * 128 * 128, static_cast<uint8_t*>(rimg));
   return finish(VDN_OK);
 }
 
