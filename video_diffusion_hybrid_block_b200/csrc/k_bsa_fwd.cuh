@@ -136,6 +136,18 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   block_rows(p.off, p.F, p.bf, b, q0, q1);
   const int qs = q0 + pair * kBsaRowsPerCta;
   if (qs >= q1) return;  // uniform over the CTA, before any resource is taken
+  // A block whose query tile count is odd leaves one CTA with a single tile.
+  // That CTA splits the key tiles instead: both warpgroups take the same
+  // query rows (Q is loaded into both Q buffers), warpgroup i the key tiles
+  // j = i, i + 2, ... into its own S_i and O_i, and warpgroup 0 combines the
+  // two partial softmaxes (m_i, l_i, O_i) at the end. Uniform over the CTA.
+  // Softmax branch alone (kMode 0), bf16 only. In the e4m3 variant each
+  // warpgroup's own running max would change which P values e4m3 rounds and
+  // how, so it keeps one running max per row; the merged epilogues keep
+  // their register budget for the readout and merge (measured: the merged
+  // kernel with split CTAs ran about 1 % slower on layouts without single
+  // tiles and gained 2 % on vda-stress).
+  const bool split = kMode == 0 && !kFp8 && qs + kTile >= q1;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t bar_q, bar_kf[2], bar_ke[2], bar_vf[2], bar_ve[2], bar_sf[2], bar_pf[2],
@@ -188,25 +200,28 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
+      // rows of the second Q buffer: the second tile, or the first again
+      // when the CTA splits its key tiles
+      const int qs1 = split ? qs : qs + kTile;
       if constexpr (kFp8) {
         // e4m3 Q tiles; the merge variant's readout also needs Q in bf16
         mbar_arrive_expect_tx(q_full, 2 * 16384 + (kMerge ? 2 * 32768 : 0));
         tma_load_3d(sQ, &tq, q_full, 0, h, qs);
-        tma_load_3d(sQ + 16384, &tq, q_full, 0, h, qs + kTile);
+        tma_load_3d(sQ + 16384, &tq, q_full, 0, h, qs1);
         if (kMerge) {
           const uint32_t sQb = base + kOffQb;
           tma_prefetch_desc(&tqb);
           tma_load_3d(sQb, &tqb, q_full, 0, h, qs);
           tma_load_3d(sQb + 16384, &tqb, q_full, 64, h, qs);
-          tma_load_3d(sQb + 32768, &tqb, q_full, 0, h, qs + kTile);
-          tma_load_3d(sQb + 49152, &tqb, q_full, 64, h, qs + kTile);
+          tma_load_3d(sQb + 32768, &tqb, q_full, 0, h, qs1);
+          tma_load_3d(sQb + 49152, &tqb, q_full, 64, h, qs1);
         }
       } else {
         mbar_arrive_expect_tx(q_full, 2 * 32768);
         tma_load_3d(sQ, &tq, q_full, 0, h, qs);
         tma_load_3d(sQ + 16384, &tq, q_full, 64, h, qs);
-        tma_load_3d(sQ + 32768, &tq, q_full, 0, h, qs + kTile);
-        tma_load_3d(sQ + 49152, &tq, q_full, 64, h, qs + kTile);
+        tma_load_3d(sQ + 32768, &tq, q_full, 0, h, qs1);
+        tma_load_3d(sQ + 49152, &tq, q_full, 64, h, qs1);
       }
       if (kMerge) {
         mbar_arrive_expect_tx(smem_u32(&bar_r), kRImageBytes);
@@ -304,13 +319,64 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       };
       bool ok = mbar_wait(q_full, 0) &&
                 mbar_wait(smem_u32(&bar_kf[0]), 0);
-      if (ok) {
+      if (split) {
+        // key tile j goes to warpgroup j & 1 through stage j & 1 (the stage
+        // the producer filled with it): S_i = Q K_j, then O_i += P_i V_j, and
+        // QK of key tile j + 2 into S_i right after (in issue order)
+        if (ok) {
+          tc_fence_after();
+          qk(0, 0);
+          umma_commit(smem_u32(&bar_ke[0]));
+          if (nkt > 1) {
+            ok = mbar_wait(smem_u32(&bar_kf[1]), 0);
+            if (ok) {
+              tc_fence_after();
+              qk(1, 1);
+              umma_commit(smem_u32(&bar_ke[1]));
+            }
+          }
+        }
+        for (int j = 0; ok && j < nkt; ++j) {
+          const int i = j & 1;
+          const uint32_t ph = (uint32_t)((j >> 1) & 1);
+          if (!mbar_wait_spin(smem_u32(&bar_vf[i]), ph) ||
+              !mbar_wait_spin(smem_u32(&bar_pf[i]), ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          pv(i, i, j >= 2);
+          umma_commit(smem_u32(&bar_ve[i]));
+          if (j + 2 < nkt) {
+            if (!mbar_wait_spin(smem_u32(&bar_kf[i]), ph ^ 1u)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            qk(i, i);
+            umma_commit(smem_u32(&bar_ke[i]));
+          }
+        }
+        if (ok && kMerge) {
+          ok = mbar_wait(smem_u32(&bar_r), 0);
+          if (ok) {
+            tc_fence_after();
+            readout(0);
+          }
+        }
+        // both commits cover every contraction issued above
+        if (ok) {
+          umma_commit(smem_u32(&bar_of[0]));
+          umma_commit(smem_u32(&bar_of[1]));
+        }
+      }
+      if (!split && ok) {
         tc_fence_after();
         qk(0, 0);
         qk(1, 0);
         umma_commit(smem_u32(&bar_ke[0]));
       }
-      for (int j = 0; ok && j < nkt; ++j) {
+      for (int j = 0; !split && ok && j < nkt; ++j) {
         const int st = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         const int st1 = (j + 1) & 1;
@@ -371,7 +437,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     if constexpr (kFp8) {
       // e4m3 scores are q8 . k8: fold the row's q scale and the head's k scale
       // into the exponent scale, the head's v scale into 1 / l
-      const int qrow = qs + tile * kTile + r;
+      const int qrow = qs + (split ? 0 : tile * kTile) + r;
       const float sq = qrow < q1 ? __ldg(p.q_scale + (int64_t)qrow * p.H + h) : 1.f;
       const float ak = __uint_as_float(__ldg(p.kv_amax + h));
       const float av = __uint_as_float(__ldg(p.kv_amax + p.H + h));
@@ -382,11 +448,15 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     float2 lacc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
     bool ok = true;
-    for (int j = 0; j < nkt; ++j) {
+    // this warpgroup's key tiles: all of them, or every other one when the
+    // CTA splits its key tiles (tile 0: j = 0, 2, ...; tile 1: j = 1, 3, ...)
+    const int nown = split ? (nkt + 1 - tile) / 2 : nkt;
+    for (int jj = 0; jj < nown; ++jj) {
+      const int j = split ? 2 * jj + tile : jj;
       int src, row0, valid;
       segs_tile(segs, j, src, row0, valid);
       // no per-tile abort poll: a failed (bounded) wait ends the loop
-      if (!mbar_wait(s_full, (uint32_t)(j & 1))) {
+      if (!mbar_wait(s_full, (uint32_t)(jj & 1))) {
         ok = false;
         *abort_v = 1;
         break;
@@ -415,7 +485,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       for (int a = 0; a < 8; ++a) mq[a] = fmaxf(mq[a], __uint_as_float(s[120 + a]));
       const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(fmax3(mq[3], mq[4], mq[5]), mq[6], mq[7]));
       const float m_tile = mx * scale;
-      if (j == 0) {
+      if (jj == 0) {
         m_use = m_tile;
       } else {
         const bool need = m_tile > m_use + 8.f;
@@ -501,9 +571,46 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     if (ok && !mbar_wait(smem_u32(&bar_of[tile]), 0)) ok = false;
     if (!ok) *abort_v = 1;
     tc_fence_after();
+    // split CTA: warpgroup 1 hands its rows' (m, l) to warpgroup 0 through
+    // the second Q buffer (idle once every contraction has completed);
+    // warpgroup 0 weights the two partial outputs by 2^(m_i - m) and adds
+    // them. Warpgroup 1's own rows lie past the block, so it stores nothing.
+    float m_fin = m_use, l_fin = l_sum, oa0 = 1.f, oa1 = 0.f;
+    const bool combine = split && tile == 0;
+    if (split) {
+      float* xch = reinterpret_cast<float*>(smem_raw + (base + kTileB - smem_u32(smem_raw)));
+      if (tile == 1) {
+        xch[r] = m_use;
+        xch[128 + r] = l_sum;  // 0 if the warpgroup had no key tile
+      }
+      named_barrier_sync(4, 256);
+      if (tile == 0) {
+        const float m1 = xch[r], l1 = xch[128 + r];
+        if (l1 > 0.f) {
+          m_fin = fmaxf(m_use, m1);
+          oa0 = ex2_approx(m_use - m_fin);
+          oa1 = ex2_approx(m1 - m_fin);
+          l_fin = l_sum * oa0 + l1 * oa1;
+        }
+      }
+    }
+    const uint32_t tO1 = tmem + lane_base + 384u;  // O_1: same lanes, next 128 columns
+    // chunk c of this row's O (already loaded from O_0): the weighted sum
+    // with O_1's chunk in a split CTA
+    auto combine_o = [&](int c, uint32_t (&o)[32]) {
+      if (!combine) return;
+      uint32_t o1[32];
+      tmem_ld32(tO1 + (uint32_t)(c * 32), o1);
+      tmem_ld_wait(o1);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float x = __uint_as_float(o[e]) * oa0;
+        o[e] = __float_as_uint(oa1 != 0.f ? fmaf(__uint_as_float(o1[e]), oa1, x) : x);
+      }
+    };
     const int row = qs + tile * kTile + r;
     const bool store = ok && row < q1;
-    const float inv = v_scale / l_sum;
+    const float inv = v_scale / l_fin;
     if (!kMerge) {
       __nv_bfloat16* dst = p.o + (int64_t)row * p.o_row_stride + (int64_t)h * p.d_store;
       // the TMEM loads are warp-collective: every thread runs them, only the
@@ -513,6 +620,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         uint32_t o[32];
         tmem_ld32(tO + (uint32_t)(c * 32), o);
         tmem_ld_wait(o);
+        combine_o(c, o);
         if (store) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -528,7 +636,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         }
       }
       if (store && p.lse != nullptr)
-        p.lse[(int64_t)h * p.N + row] = (m_use + __log2f(l_sum)) * 0.69314718055994531f;
+        p.lse[(int64_t)h * p.N + row] = (m_fin + __log2f(l_fin)) * 0.69314718055994531f;
     } else {
       // gated merge of O / l with RMSNorm(o_lin); o_lin sits in the S_i columns
       const int64_t gi = (int64_t)row * p.H + h;
@@ -557,6 +665,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
             uint32_t x[32];
             tmem_ld32((pass == 0 ? tO : tS) + (uint32_t)(c * 32), x);
             tmem_ld_wait(x);
+            if (pass == 0) combine_o(c, x);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int c0 = c * 32 + u * 8;
@@ -599,6 +708,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         tmem_ld32(tS + (uint32_t)(c * 32), z);
         tmem_ld_wait(o);
         tmem_ld_wait(z);
+        combine_o(c, o);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int c0 = c * 32 + u * 8;
